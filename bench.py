@@ -1,0 +1,397 @@
+#!/usr/bin/env python
+"""Benchmark of the AdaFuse decode-step hot path on B200.
+
+One step = one token of the decode switch sequence: pre-gate the token's
+first-layer hidden state (one top-2 routing decision), then one fused switch
+launch that un-merges the previous token's experts and merges this token's
+into every LoRA-targeted weight of every layer, in place.
+
+value   = W bytes read + written by the switches / device time (GB/s), summed
+          over ranks (each rank is an independent replica: the switch of one
+          model has no exchange step).
+e2e     = the same through the public API with the step's input (the token's
+          hidden state) copied from pinned host memory and the step's result
+          (its route record) copied back, inside the timed region.
+roofline= the switch kernel's algorithmic W bytes / its CUDA-event duration,
+          against the measured HBM copy bandwidth.
+
+`--impl reference` times the fp64 CPU oracle on the host cores instead, on a
+bounded row sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "adapter-switch latency & HBM GB/s (W read+write) at Llama-2-7B shape, % of peak"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="7b")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="override the layer count (small cases for ncu captures)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--traffic-gb", type=float, default=None,
+                    help="ncu dram bytes (read+write) of one switch launch, GB")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9 and parts[1].isdigit():
+                    rows.append(parts)
+        except Exception:
+            pass
+        finally:
+            try:
+                os.unlink(self.path)
+            except Exception:
+                pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [int(r[1]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": int(rows[0][2]),
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())
+                if any(r[3].replace(".", "").isdigit() for r in rows) else None}
+
+
+# --------------------------------------------------------------------------
+# CPU oracle timing (the reported baseline; never the product path)
+
+_ORACLE_MODELS = {}
+
+
+def oracle_rate(cfg, target_s=10.0, seed_layers=1):
+    """fp64 oracle switch on a bounded row sample of layer 0 of the workload.
+    Returns (W GB/s equivalent, threads, sample description, elapsed s)."""
+    import numpy as np
+    import torch
+
+    import oracle
+    from weight_merge_b200 import workloads as wl
+
+    oracle.build()
+    key = (cfg.name, seed_layers)
+    if key not in _ORACLE_MODELS:
+        _ORACLE_MODELS[key] = wl.make_model(wl.scaled(cfg, n_layers=seed_layers), device="cpu")
+    m = _ORACLE_MODELS[key]
+    bits = lambda t: t.view(torch.int16).numpy().view(np.uint16)
+    A = [bits(a) for a in m.A]
+    B = [bits(b) for b in m.B]
+    E = cfg.n_experts
+    prev = (np.array([0, 1], np.int32), np.array([0.6, 0.4], np.float32))
+    cur = (np.array([2, 3 % E], np.int32), np.array([0.7, 0.3], np.float32))
+
+    def run(rows_per_target):
+        elems = 0
+        t0 = time.perf_counter()
+        for i, w in enumerate(m.W):
+            out = w.shape[0]
+            rows = np.arange(min(rows_per_target, out), dtype=np.int64)
+            oracle.switch_rows(bits(w[: len(rows)]), rows, out, A[i], B[i], cfg.scale, prev, cur)
+            elems += len(rows) * w.shape[1]
+        return elems, time.perf_counter() - t0
+
+    e0, t0 = run(8)
+    rate = e0 / max(t0, 1e-6)
+    per_row = e0 / 8
+    rows = int(max(8, min(4096, target_s * rate / per_row)))
+    elems, dt = run(rows)
+    gbs = elems * 4 / dt / 1e9
+    desc = (f"fp64 oracle switch (4 experts: 2 out, 2 in) on the first {rows} rows of each of "
+            f"the {len(cfg.targets)} targets of one layer, {elems/1e6:.1f} M W elements; "
+            f"W-bytes rate extrapolates to a full switch")
+    return gbs, oracle.num_threads(), desc, dt, elems
+
+
+# --------------------------------------------------------------------------
+# the reference arm: the oracle, on the host cores
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from weight_merge_b200 import workloads as wl
+    cfg = wl.CONFIGS[args.config]
+    # each step: a bounded sample (~2 s) of one switch
+    times = []
+    gbs_all = []
+    desc = threads = None
+    for k in range(args.warmup + args.steps):
+        gbs, threads, desc, dt, elems = oracle_rate(cfg, target_s=2.0)
+        if k >= args.warmup:
+            times.append(dt)
+            gbs_all.append(gbs)
+    value = statistics.mean(gbs_all)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1000 * statistics.mean(times), 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{cfg.name}: {cfg.n_layers} layers, d={cfg.d}, "
+                               f"E={cfg.n_experts}, r={cfg.rank}, row sample of one layer"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads,
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------
+# our arm
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from weight_merge_b200 import binding as B
+    from weight_merge_b200 import workloads as wl
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.cuda.current_device()
+
+    cfg = wl.CONFIGS[args.config]
+    if args.layers:
+        cfg = wl.scaled(cfg, n_layers=args.layers)
+    model = wl.make_model(cfg, device="cuda")
+    sw = B.Switcher(model.W, model.A, model.B, cfg.n_layers, len(cfg.targets), cfg.n_experts,
+                    cfg.rank, cfg.alpha, device=dev, names=[t.name for t in cfg.targets])
+    T = cfg.n_tokens
+    h = wl.make_hidden(cfg, T=T, device="cuda")
+    routes = torch.zeros((T, 4), dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+    sh = stream.cuda_stream
+    w_bytes = cfg.w_bytes_per_switch()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def step(k, prev_t):
+        t = k % T
+        sw.pregate(h[t:t + 1], model.Wr, routes[t:t + 1], sh)
+        sw.switch(B.Switcher.route_ptr(routes, prev_t), B.Switcher.route_ptr(routes, t), sh)
+        return t
+
+    # warm-up
+    prev_t = None
+    for k in range(args.warmup):
+        prev_t = step(k, prev_t)
+    torch.cuda.synchronize()
+    assert sw.status(sh) == 0
+
+    # timed region: K steps, events around every switch launch for the roofline
+    n_ev = args.steps
+    sw_start = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    sw_end = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    st_start = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    t_begin = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        t_begin.record(stream)
+        for k in range(args.steps):
+            kk = args.warmup + k
+            t = kk % T
+            st_start[k].record(stream)
+            sw.pregate(h[t:t + 1], model.Wr, routes[t:t + 1], sh)
+            sw_start[k].record(stream)
+            sw.switch(B.Switcher.route_ptr(routes, prev_t), B.Switcher.route_ptr(routes, t), sh)
+            sw_end[k].record(stream)
+            prev_t = t
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    clocks = clk.summary()
+    assert sw.status(sh) == 0
+    total_ms = t_begin.elapsed_time(t_end)
+    sw_ms = [a.elapsed_time(b) for a, b in zip(sw_start, sw_end)]
+    step_ms = [st_start[k].elapsed_time(st_start[k + 1]) for k in range(n_ev - 1)]
+    step_ms.append(st_start[-1].elapsed_time(t_end))
+
+    # identity steps (prev == cur bit-identical) move no W bytes
+    r_np = routes.cpu().numpy()
+    n_real = 0
+    p = (args.warmup - 1) % T if args.warmup > 0 else None
+    for k in range(args.steps):
+        t = (args.warmup + k) % T
+        if p is None or not np.array_equal(r_np[p], r_np[t]):
+            n_real += 1
+        p = t
+
+    # max over ranks
+    tm = torch.tensor([total_ms, float(n_real)], dtype=torch.float64, device="cuda")
+    if world > 1:
+        mx = tm.clone()
+        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+        tot_real = tm[1:].clone()
+        dist.all_reduce(tot_real, op=dist.ReduceOp.SUM)
+        max_ms, all_real = float(mx[0]), float(tot_real[0])
+    else:
+        max_ms, all_real = total_ms, float(n_real)
+    value = all_real * w_bytes / (max_ms / 1000.0) / 1e9
+
+    # e2e through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        h_host = h.cpu().pin_memory()
+        r_host = torch.zeros((1, 4), dtype=torch.int32).pin_memory()
+        h_dev = torch.empty((1, cfg.d), dtype=torch.float32, device="cuda")
+        ev0 = torch.cuda.Event(enable_timing=True)
+        ev1 = torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        pe = prev_t
+        for k in range(args.steps):
+            t = (args.warmup + args.steps + k) % T
+            h_dev.copy_(h_host[t:t + 1], non_blocking=True)
+            sw.pregate(h_dev, model.Wr, routes[t:t + 1], sh)
+            sw.switch(B.Switcher.route_ptr(routes, pe), B.Switcher.route_ptr(routes, t), sh)
+            r_host.copy_(routes[t:t + 1], non_blocking=True)
+            pe = t
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e_ms = ev0.elapsed_time(ev1)
+        et = torch.tensor([e_ms], dtype=torch.float64, device="cuda")
+        if world > 1:
+            dist.all_reduce(et, op=dist.ReduceOp.MAX)
+        e2e = {"value": round(world * args.steps * w_bytes / (float(et[0]) / 1000) / 1e9, 2),
+               "unit": "GB/s", "h2d_bytes_per_step": cfg.d * 4, "d2h_bytes_per_step": 16}
+
+    peak, peak_kind = measured_peaks()
+    sw_avg = statistics.mean(sw_ms)
+    achieved = w_bytes / (sw_avg / 1000.0) / 1e9
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gbs, threads, desc, dt, elems = oracle_rate(cfg, target_s=10.0)
+        cpu = {"value": round(gbs, 5), "unit": "GB/s", "cores": threads, "kind": "oracle",
+               "sample": desc}
+
+    if rank == 0:
+        sw_sorted = sorted(sw_ms)
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(max_ms / args.steps, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded random weights and hidden states)",
+            "config": {
+                "workload": f"{cfg.name}: Llama-2-7B-shaped, {cfg.n_layers} layers x "
+                            f"{len(cfg.targets)} targets (q,k,v,o {cfg.d}x{cfg.d}; gate,up "
+                            f"{cfg.targets[4].out}x{cfg.d}; down {cfg.d}x{cfg.targets[6].inn}), "
+                            f"E={cfg.n_experts}, r={cfg.rank}, alpha={cfg.alpha:g}, top-2, "
+                            f"{T}-token decode switch sequence",
+                "w_bytes_per_switch": w_bytes,
+                "l2": "inputs larger than L2 (W read+write per switch >> 126 MB), no flush",
+                "parallelism": f"replicas x{world}",
+            },
+            "switch_ms_p50": round(sw_sorted[len(sw_sorted) // 2], 4),
+            "switch_ms_p90": round(sw_sorted[min(len(sw_sorted) - 1, int(0.9 * len(sw_sorted)))], 4),
+            "step_ms_p50": round(sorted(step_ms)[len(step_ms) // 2], 4),
+            "switches_per_s": round(world * args.steps / (max_ms / 1000.0), 3),
+            "identity_steps": args.steps - n_real,
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                         "unit": "GB/s", "frac": round(achieved / peak, 4),
+                         "peak_kind": peak_kind,
+                         "traffic": (round(args.traffic_gb * 1e9) if args.traffic_gb else None),
+                         "kernel": "switch_mma_kernel"},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": 2 * args.steps,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    sw.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,193 @@
+/*
+ * adafuse.h -- C ABI of the AdaFuse adapter switch for NVIDIA B200 (sm_100a).
+ *
+ * What the library computes (page title "AdaFuse: Accelerating Dynamic
+ * Adapter Inference via Token-Level Pre-Gating and Fused Kernel
+ * Optimization"):
+ *
+ *   adafuse_pregate   token-level pre-gating: ONE top-2 routing decision per
+ *                     token, made from the hidden state entering the first
+ *                     layer, and applied to every adapter layer
+ *                     (gist.science technical summary, section 2-ga, items
+ *                     1-3; shd-paper.top summary, English abstract).
+ *   adafuse_switch    the fused adapter switch: in ONE kernel launch, for
+ *                     every layer and every LoRA-targeted weight, remove the
+ *                     previous token's gated experts and merge the current
+ *                     token's, in place:
+ *                       W <- W - s*sum_{e in prev} g_e B_e A_e
+ *                              + s*sum_{e in cur}  g_e B_e A_e
+ *                     (gist.science technical summary, section 2-na: the SGMM
+ *                     "segmented gather matrix multiplication" kernel,
+ *                     concatenated adapter matrices, in-place update,
+ *                     prefetch buffer).
+ *   adafuse_switch_batch_layers   the same switch restricted to a contiguous
+ *                     range of layers (for pipelining against the forward).
+ *
+ * Numerics: W is bf16; each W element is updated as
+ *   W <- bf16_round_nearest_even(float(W) + dW)
+ * with dW = sum_e c_e * (B_e A_e), the products accumulated in fp32 and the
+ * per-expert coefficients c_e = s*(g_cur(e) - g_prev(e)) applied in fp32.
+ * One rounding per element per switch.  s = alpha / rank.
+ *
+ * Layouts (all row-major, all device memory unless stated):
+ *   W  [out, in]        bf16   the backbone weight, updated in place
+ *   A  [E, rank, in]    bf16   LoRA down-projections of the E experts
+ *   B  [E, out, rank]   bf16   LoRA up-projections of the E experts
+ *   h  [T, d]           fp32   hidden states entering the first layer
+ *   Wr [d, E]           fp32   router weight
+ *   route [T]           adafuse_route (16 bytes each)
+ *
+ * Ownership: the caller owns every buffer named above, keeps it alive and
+ * in place for the life of the context, and must not write W while a switch
+ * on it is in flight.  The library owns the context, its device-side
+ * segment table and its device status word.  The library keeps no copy of W.
+ *
+ * Errors: every call returns ADAFUSE_OK (0) or a negative code.  Calls that
+ * take a stream are asynchronous with respect to the host; host-side
+ * argument errors are reported before anything is launched.  Problems only
+ * the device can see (an expert index outside [-1, E), a non-finite gate in
+ * a route) make the switch write NOTHING and raise a bit in the context's
+ * device status word (read it with adafuse_get_device_status).  No C++
+ * exception crosses this boundary.  A context may be used from one host
+ * thread and one stream at a time.
+ */
+#ifndef ADAFUSE_H_
+#define ADAFUSE_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ADAFUSE_API __attribute__((visibility("default")))
+#else
+#define ADAFUSE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- return codes ------------------------------------------------------- */
+#define ADAFUSE_OK                     0
+#define ADAFUSE_ERR_INVALID_ARG       -1  /* NULL pointer, bad count, misaligned pointer */
+#define ADAFUSE_ERR_UNSUPPORTED_SHAPE -2  /* dims not multiples of 8, rank outside [1,64], E outside [1,64] */
+#define ADAFUSE_ERR_CUDA              -3  /* a CUDA runtime call failed (see adafuse_last_error) */
+#define ADAFUSE_ERR_DEVICE_FAULT      -4  /* the device status word is non-zero */
+#define ADAFUSE_ERR_UNSUPPORTED_DEVICE -5 /* not a compute-capability 10.0 (B200-class) GPU */
+#define ADAFUSE_ERR_OUT_OF_MEMORY     -6  /* host or device allocation failed */
+
+/* ---- device status word bits (adafuse_get_device_status) ---------------- */
+#define ADAFUSE_STATUS_BAD_EXPERT   0x1   /* a route held an index outside [-1, E) */
+#define ADAFUSE_STATUS_BAD_GATE     0x2   /* a route held a non-finite gate on a used slot */
+
+/* One token's routing decision: the two chosen experts and their gates.
+ * idx[j] == -1 marks an empty slot (its gate is ignored).  adafuse_pregate
+ * writes gate[0] >= gate[1], gate[0] + gate[1] == 1 (up to rounding). */
+typedef struct adafuse_route {
+    int32_t idx[2];
+    float gate[2];
+} adafuse_route;
+
+/* One LoRA-targeted weight of one layer (for example q_proj of layer 7).
+ *   out, in  W's shape; both multiples of 8.
+ *   W        device pointer, [out, in] bf16, 16-byte aligned, updated in place.
+ *   A        device pointer, [E, rank, in] bf16, 16-byte aligned.
+ *   B        device pointer, [E, out, rank] bf16, 16-byte aligned.
+ *   name     optional label (may be NULL); not copied, not used by kernels. */
+typedef struct adafuse_target {
+    const char* name;
+    int64_t out;
+    int64_t in;
+    void* W;
+    const void* A;
+    const void* B;
+} adafuse_target;
+
+/* The adapter-carrying model.  targets has n_layers * n_targets entries,
+ * layer-major: targets[l * n_targets + k] is target k of layer l.
+ * 1 <= n_experts <= 64, 1 <= rank <= 64, alpha finite; s = alpha / rank. */
+typedef struct adafuse_desc {
+    int32_t n_layers;
+    int32_t n_targets;
+    int32_t n_experts;
+    int32_t rank;
+    float alpha;
+    const adafuse_target* targets;
+} adafuse_desc;
+
+typedef struct adafuse_ctx adafuse_ctx;
+
+/* Validate the model, build the device-side segment table (the list of
+ * disjoint 128x128 W tiles of every (layer, target), layer-major) and the
+ * per-weight descriptors, and copy them to `device`.  Not on the hot path.
+ * Returns INVALID_ARG / UNSUPPORTED_SHAPE / UNSUPPORTED_DEVICE / CUDA /
+ * OUT_OF_MEMORY without creating anything.  *out receives the context. */
+ADAFUSE_API int adafuse_create(adafuse_ctx** out, const adafuse_desc* desc, int device);
+
+/* Free the context and its device memory.  The caller must make sure no
+ * call using it is still in flight.  NULL is accepted (no-op). */
+ADAFUSE_API int adafuse_destroy(adafuse_ctx* ctx);
+
+/* Token-level pre-gating (section 2-ga): for each of T tokens,
+ *   z_e = sum_i h[t,i] * Wr[i,e]  (fp32; every column reduced in the same
+ *         order, so equal columns give bitwise-equal logits),
+ *   the two experts first under (z descending, index ascending),
+ *   gates = softmax over all E renormalised over the two picks, computed
+ *         in the equal closed form g0 = 1/(1+x), g1 = x/(1+x),
+ *         x = exp(z1 - z0),
+ * written to route[t].  E comes from the context.  With E == 1 the route is
+ * {0, -1} with gates {1, 0}.  h, Wr, route are device pointers; h and route
+ * 16-byte aligned, Wr 4-byte aligned, d a multiple of 4 and d >= 1; T == 0
+ * is a no-op.
+ * Non-finite h gives an unspecified route (the switch rejects non-finite
+ * gates).  One kernel launch on `stream` (a cudaStream_t, NULL = legacy
+ * default stream). */
+ADAFUSE_API int adafuse_pregate(adafuse_ctx* ctx, const float* h, int64_t T, int64_t d,
+                    const float* Wr, adafuse_route* route, void* stream);
+
+/* The fused adapter switch (section 2-na) over ALL layers and targets, one
+ * kernel launch on `stream`.  prev / cur are 16-byte aligned device
+ * pointers to ONE route each, or NULL for "no experts" (prev == NULL: first
+ * token, or a static
+ * pre-merge; cur == NULL: full unmerge).  Per expert e in prev U cur the
+ * coefficient is c_e = s*(g_cur(e) - g_prev(e)) (an absent side counts 0);
+ * experts with c_e == 0 are dropped, so prev == cur (same indices, bitwise
+ * equal gates) launches work that writes nothing and leaves W bit-identical.
+ * The route records are read on the device: no host synchronisation. */
+ADAFUSE_API int adafuse_switch(adafuse_ctx* ctx, const adafuse_route* prev,
+                   const adafuse_route* cur, void* stream);
+
+/* As adafuse_switch, restricted to layers [layer_begin, layer_begin +
+ * n_layers).  n_layers == 0 is a no-op; a range outside [0, L) is
+ * INVALID_ARG.  Running it over a partition of [0, L) equals one
+ * adafuse_switch. */
+ADAFUSE_API int adafuse_switch_batch_layers(adafuse_ctx* ctx, int32_t layer_begin,
+                                int32_t n_layers, const adafuse_route* prev,
+                                const adafuse_route* cur, void* stream);
+
+/* Synchronise `stream`, read the device status word into *status, then
+ * clear it.  Returns ADAFUSE_ERR_DEVICE_FAULT when the word was non-zero,
+ * ADAFUSE_OK otherwise. */
+ADAFUSE_API int adafuse_get_device_status(adafuse_ctx* ctx, void* stream, int32_t* status);
+
+/* Host-only introspection (no device work): the segment table the context
+ * would build for `desc`, as n entries of 4 int32 {layer, target, row0,
+ * col0}, tile size 128x128.  With entries == NULL only *count is written.
+ * capacity counts entries.  Returns INVALID_ARG if capacity is too small. */
+ADAFUSE_API int adafuse_segment_table(const adafuse_desc* desc, int32_t* entries,
+                          int64_t capacity, int64_t* count);
+
+/* Tile edge of the segment table (128). */
+ADAFUSE_API int adafuse_tile_size(void);
+
+/* Human-readable text for a return code (static storage). */
+ADAFUSE_API const char* adafuse_strerror(int code);
+
+/* Text of the last CUDA error this host thread saw in the library (static
+ * thread-local storage, "" when none). */
+ADAFUSE_API const char* adafuse_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ADAFUSE_H_ */

@@ -1,0 +1,119 @@
+"""Host-side checks of the C-ABI library: it loads, exports every declared
+symbol, rejects bad arguments before touching the GPU, and builds a segment
+table whose tiles cover every W element exactly once.  No GPU needed."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from weight_merge_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from weight_merge_b200 import build
+    build.build()
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "adafuse.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(adafuse_\w+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    syms = declared_symbols()
+    assert len(syms) >= 10
+    L = ctypes.CDLL(B.library_path())
+    for s in syms:
+        assert hasattr(L, s), s
+
+
+def test_tile_size_and_strerror():
+    assert B.adafuse_tile_size() == 128
+    assert B.adafuse_strerror(0) == "ok"
+    assert "invalid" in B.adafuse_strerror(B.ADAFUSE_ERR_INVALID_ARG)
+    assert B.adafuse_last_error() == ""
+
+
+def _desc(shapes, n_layers, E=4, r=8, alpha=16.0, ptr=16):
+    ts = []
+    for l in range(n_layers):
+        for k, (o, i) in enumerate(shapes):
+            ts.append((f"t{k}", o, i, ptr, ptr, ptr))
+    return B.make_desc(n_layers, len(shapes), E, r, alpha, ts)
+
+
+@pytest.mark.parametrize("shapes,L", [
+    ([(256, 256), (256, 256)], 2),
+    ([(4096, 4096), (11008, 4096), (4096, 11008)], 2),
+    ([(200, 136), (8, 8), (1024, 4096), (136, 264)], 3),
+])
+def test_segment_table_covers_each_element_once(shapes, L):
+    d = _desc(shapes, L)
+    tab = B.adafuse_segment_table(d)
+    T = B.adafuse_tile_size()
+    # layer-major, then target, then row / col tile
+    keys = [tuple(x) for x in tab]
+    assert keys == sorted(keys)
+    for l in range(L):
+        for k, (o, i) in enumerate(shapes):
+            sel = tab[(tab[:, 0] == l) & (tab[:, 1] == k)]
+            assert len(sel) == -(-o // T) * -(-i // T)
+            cover = np.zeros((o, i), dtype=np.int32)
+            for _, _, r0, c0 in sel:
+                assert r0 % T == 0 and c0 % T == 0 and r0 < o and c0 < i
+                cover[r0:r0 + T, c0:c0 + T] += 1
+            assert cover.min() == 1 and cover.max() == 1
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(shapes=[(100, 64)]), B.ADAFUSE_ERR_UNSUPPORTED_SHAPE),
+    (dict(shapes=[(64, 60)]), B.ADAFUSE_ERR_UNSUPPORTED_SHAPE),
+    (dict(r=0), B.ADAFUSE_ERR_UNSUPPORTED_SHAPE),
+    (dict(r=65), B.ADAFUSE_ERR_UNSUPPORTED_SHAPE),
+    (dict(E=0), B.ADAFUSE_ERR_UNSUPPORTED_SHAPE),
+    (dict(E=65), B.ADAFUSE_ERR_UNSUPPORTED_SHAPE),
+    (dict(alpha=float("nan")), B.ADAFUSE_ERR_INVALID_ARG),
+    (dict(shapes=[(0, 64)]), B.ADAFUSE_ERR_INVALID_ARG),
+])
+def test_bad_descriptors_rejected_on_host(bad, code):
+    kw = dict(shapes=[(64, 64)], L=1, E=4, r=8, alpha=16.0)
+    kw.update(bad)
+    d = _desc(kw["shapes"], kw["L"], kw["E"], kw["r"], kw["alpha"])
+    n = ctypes.c_int64()
+    assert B.lib().adafuse_segment_table(ctypes.byref(d), None, 0, ctypes.byref(n)) == code
+    h = ctypes.c_void_p()
+    assert B.lib().adafuse_create(ctypes.byref(h), ctypes.byref(d), 0) == code
+    assert h.value is None
+
+
+def test_create_rejects_null_and_misaligned_pointers():
+    h = ctypes.c_void_p()
+    assert B.lib().adafuse_create(ctypes.byref(h), None, 0) == B.ADAFUSE_ERR_INVALID_ARG
+    d = _desc([(64, 64)], 1, ptr=0)
+    assert B.lib().adafuse_create(ctypes.byref(h), ctypes.byref(d), 0) == B.ADAFUSE_ERR_INVALID_ARG
+    d = _desc([(64, 64)], 1, ptr=24)
+    assert B.lib().adafuse_create(ctypes.byref(h), ctypes.byref(d), 0) == B.ADAFUSE_ERR_INVALID_ARG
+
+
+def test_calls_on_null_context_are_invalid():
+    L = B.lib()
+    assert L.adafuse_switch(None, None, None, None) == B.ADAFUSE_ERR_INVALID_ARG
+    assert L.adafuse_switch_batch_layers(None, 0, 1, None, None, None) == B.ADAFUSE_ERR_INVALID_ARG
+    assert L.adafuse_pregate(None, None, 1, 8, None, None, None) == B.ADAFUSE_ERR_INVALID_ARG
+    st = ctypes.c_int32()
+    assert L.adafuse_get_device_status(None, None, ctypes.byref(st)) == B.ADAFUSE_ERR_INVALID_ARG
+    assert L.adafuse_destroy(None) == B.ADAFUSE_OK
+
+
+def test_segment_table_capacity_checked():
+    d = _desc([(256, 256)], 1)
+    n = ctypes.c_int64()
+    buf = (ctypes.c_int32 * 8)()
+    assert B.lib().adafuse_segment_table(ctypes.byref(d), buf, 2, ctypes.byref(n)) == B.ADAFUSE_ERR_INVALID_ARG
+    assert n.value == 4

@@ -1,0 +1,326 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 CPU oracle.
+
+Bars (AdaFuse pages, gist.science technical summary sections 2-ga / 2-na,
+with the tolerances of the build's contract):
+  * expert indices bit-exact (ties to the lower index; a token whose fp64
+    order is within the fp32 rounding bound may differ and is counted),
+  * gates within 1e-5 relative,
+  * every checked W element within 1 bf16 step of the oracle, which starts
+    from the GPU's own pre-switch W (lockstep, so rounding drift over many
+    switches does not accumulate into the comparison).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from weight_merge_b200 import binding as Bnd
+from weight_merge_b200 import workloads as wl
+
+from .util import (bits, make_routes, pregate_consistent, route_tuple, routes_to_np,
+                   ulp_dist)
+
+pytestmark = pytest.mark.gpu
+
+GATE_RTOL = 1e-5
+MAX_ULP = 1
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from weight_merge_b200 import build
+    build.build()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    oracle.build()
+
+
+def stream():
+    return torch.cuda.current_stream().cuda_stream
+
+
+def make_switcher(model: wl.Model) -> Bnd.Switcher:
+    c = model.cfg
+    return Bnd.Switcher(model.W, model.A, model.B, c.n_layers, len(c.targets), c.n_experts,
+                        c.rank, c.alpha, device=torch.cuda.current_device(),
+                        names=[t.name for t in c.targets])
+
+
+def host_ab(model):
+    return [bits(a) for a in model.A], [bits(b) for b in model.B]
+
+
+def check_pregate(sw, h, Wr, E):
+    T, d = h.shape
+    routes = torch.zeros((T, 4), dtype=torch.int32, device="cuda")
+    sw.pregate(h, Wr, routes, stream())
+    torch.cuda.synchronize()
+    got = routes_to_np(routes)
+    h_np, Wr_np = h.cpu().numpy(), Wr.cpu().numpy()
+    idx_ref, gate_ref, z = oracle.pregate(h_np, Wr_np, return_logits=True)
+    exact, amb = pregate_consistent(got[:, :2], idx_ref, z, h_np, Wr_np)
+    match = np.all(got[:, :2] == idx_ref, axis=1)
+    g = got[:, 2:].view(np.float32)
+    np.testing.assert_allclose(g[match], gate_ref[match], rtol=GATE_RTOL, atol=0)
+    return routes, got, amb
+
+
+def lockstep(sw, model, routes_np, routes_dev, steps, rows_of, A_h, B_h):
+    """Run switches (prev_t, cur_t) -- None = no route -- and compare the rows
+    rows_of(pair_index, out) of every weight with the oracle after each."""
+    cfg = model.cfg
+    nt = len(cfg.targets)
+    worst = 0
+    for (p, c) in steps:
+        sel = [rows_of(i, w.shape[0]) for i, w in enumerate(model.W)]
+        before = [bits(w[torch.as_tensor(r, device="cuda")]) for w, r in zip(model.W, sel)]
+        sw.switch(Bnd.Switcher.route_ptr(routes_dev, p), Bnd.Switcher.route_ptr(routes_dev, c),
+                  stream())
+        torch.cuda.synchronize()
+        assert sw.status(stream()) == 0
+        prev = route_tuple(routes_np, p) if p is not None else None
+        cur = route_tuple(routes_np, c) if c is not None else None
+        for i, w in enumerate(model.W):
+            after = bits(w[torch.as_tensor(sel[i], device="cuda")])
+            want = oracle.switch_rows(before[i], sel[i], w.shape[0], A_h[i], B_h[i], cfg.scale,
+                                      prev, cur)
+            d = ulp_dist(after, want)
+            if d.max() > MAX_ULP:
+                bad = np.argwhere(d > MAX_ULP)[0]
+                raise AssertionError(
+                    f"switch {(p, c)} layer {i // nt} target {cfg.targets[i % nt].name} "
+                    f"row {sel[i][bad[0]]} col {bad[1]}: gpu {after[tuple(bad)]:#06x} "
+                    f"oracle {want[tuple(bad)]:#06x} ({d.max()} steps)")
+            worst = max(worst, int(d.max()))
+    return worst
+
+
+def all_rows(i, out):
+    return np.arange(out, dtype=np.int64)
+
+
+# --------------------------------------------------------------------------
+# pre-gating
+
+@pytest.mark.parametrize("T,d,E", [(1, 4, 1), (1, 4096, 8), (7, 256, 4), (64, 4096, 8),
+                                   (33, 5120, 16), (5, 264, 33), (9, 128, 64), (300, 512, 3)])
+def test_pregate_matches_oracle(T, d, E):
+    cfg = wl.custom("p", 1, [("q", 8, 8)], n_experts=E, rank=8, alpha=16, n_tokens=T, d=d)
+    model = wl.make_model(cfg, device="cuda", seed=11 + E)
+    g = torch.Generator(device="cuda").manual_seed(100 + T)
+    h = torch.randn((T, d), generator=g, device="cuda")
+    Wr = torch.randn((d, E), generator=g, device="cuda") * 0.05
+    sw = make_switcher(model)
+    _, got, amb = check_pregate(sw, h, Wr, E)
+    assert len(amb) <= max(1, T // 50)
+    if E == 1:
+        assert np.all(got[:, 1] == -1)
+
+
+def test_pregate_duplicate_columns_tie_exactly():
+    T, d, E = 64, 4096, 8
+    cfg = wl.custom("p", 1, [("q", 8, 8)], n_experts=E, rank=8, alpha=16, n_tokens=T, d=d)
+    sw = make_switcher(wl.make_model(cfg, device="cuda"))
+    g = torch.Generator(device="cuda").manual_seed(5)
+    h = torch.randn((T, d), generator=g, device="cuda").abs()
+    Wr = torch.randn((d, E), generator=g, device="cuda") * 0.05
+    Wr[:, 2] = Wr[:, 2].abs() + 0.5
+    Wr[:, 6] = Wr[:, 2]
+    routes = torch.zeros((T, 4), dtype=torch.int32, device="cuda")
+    sw.pregate(h, Wr, routes, stream())
+    got = routes_to_np(routes)
+    assert np.all(got[:, 0] == 2) and np.all(got[:, 1] == 6)
+    assert np.all(got[:, 2:].view(np.float32) == np.float32(0.5))
+
+
+# --------------------------------------------------------------------------
+# the switch, small sizes, every element
+
+def test_tiny_sequence_lockstep_all_elements():
+    cfg = wl.CONFIGS["tiny"]
+    model = wl.make_model(cfg, device="cuda")
+    sw = make_switcher(model)
+    h = wl.make_hidden(cfg, device="cuda")
+    routes, routes_np, amb = check_pregate(sw, h, model.Wr, cfg.n_experts)
+    assert len(amb) == 0
+    A_h, B_h = host_ab(model)
+    steps = [(None, 0)] + [(t - 1, t) for t in range(1, cfg.n_tokens)] + [(cfg.n_tokens - 1, None)]
+    lockstep(sw, model, routes_np, routes, steps, all_rows, A_h, B_h)
+
+
+RAGGED = [("a", 200, 136), ("b", 8, 8), ("c", 264, 392), ("d", 128, 256), ("e", 136, 8)]
+
+
+@pytest.mark.parametrize("E,r", [(1, 1), (3, 3), (4, 4), (5, 8), (16, 12), (4, 16), (6, 24),
+                                 (3, 32), (4, 40), (5, 64)])
+def test_ragged_shapes_every_rank_class(E, r):
+    cfg = wl.custom("ragged", 2, RAGGED, n_experts=E, rank=r, alpha=2.0 * r, n_tokens=6,
+                    d=136)
+    model = wl.make_model(cfg, device="cuda", seed=1000 + 7 * r + E)
+    sw = make_switcher(model)
+    rng = np.random.default_rng(r * 31 + E)
+    T = 6
+    idx = rng.integers(0, E, size=(T, 2)).astype(np.int32)
+    if E > 1:
+        idx[2] = [idx[1][0], (idx[1][0] + 1) % E]   # token 2 shares an expert with token 1
+    idx[3, 1] = -1                                # an empty slot
+    if E > 1:
+        idx[4] = [idx[4][0], idx[4][0]]           # the same expert twice
+    gate = rng.uniform(0.05, 1.0, size=(T, 2)).astype(np.float32)
+    routes = make_routes(idx, gate)
+    routes_np = routes_to_np(routes)
+    A_h, B_h = host_ab(model)
+    steps = [(None, 0), (0, 1), (1, 2), (2, 3), (3, 4), (4, 5), (5, None)]
+    lockstep(sw, model, routes_np, routes, steps, all_rows, A_h, B_h)
+
+
+def _small_model(seed=3, E=4, r=8):
+    cfg = wl.custom("s", 3, [("q", 256, 384), ("o", 384, 256)], n_experts=E, rank=r,
+                    alpha=2.0 * r, n_tokens=4, d=384)
+    return wl.make_model(cfg, device="cuda", seed=seed)
+
+
+def test_identity_switches_leave_w_bit_identical():
+    model = _small_model()
+    sw = make_switcher(model)
+    W0 = [bits(w) for w in model.W]
+    idx = np.array([[1, 2], [2, 1], [0, 3]], dtype=np.int32)
+    gate = np.array([[0.8, 0.2], [0.2, 0.8], [0.0, 0.0]], dtype=np.float32)
+    routes = make_routes(idx, gate)
+    p = lambda t: Bnd.Switcher.route_ptr(routes, t)
+    for prev, cur in [(p(0), p(0)), (p(0), p(1)), (None, None), (None, p(2)), (p(2), None)]:
+        sw.switch(prev, cur, stream())
+    torch.cuda.synchronize()
+    assert sw.status(stream()) == 0
+    for w, w0 in zip(model.W, W0):
+        assert np.array_equal(bits(w), w0)
+
+
+def test_merge_then_unmerge_restores_within_rounding():
+    model = _small_model(seed=4)
+    sw = make_switcher(model)
+    W0 = [bits(w) for w in model.W]
+    routes = make_routes(np.array([[0, 3]], np.int32), np.array([[0.55, 0.45]], np.float32))
+    sw.switch(None, Bnd.Switcher.route_ptr(routes, 0), stream())
+    W1 = [bits(w) for w in model.W]
+    sw.switch(Bnd.Switcher.route_ptr(routes, 0), None, stream())
+    torch.cuda.synchronize()
+    for w, w0, w1 in zip(model.W, W0, W1):
+        w2 = bits(w)
+        assert ulp_dist(w1, w0).max() > 0
+        # two roundings of at most half a step each (see the oracle pin)
+        f = lambda b: (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        e = lambda b: np.ldexp(1.0, np.where(((b >> 7) & 0xFF) == 0, -133,
+                                             ((b.astype(np.int32) >> 7) & 0xFF) - 134))
+        assert np.all(np.abs(f(w2) - f(w0)) <= 0.5 * e(w1) + 0.5 * e(w2) + 1e-30)
+
+
+def test_layer_ranges_equal_one_full_switch():
+    m1, m2 = _small_model(seed=9), _small_model(seed=9)
+    s1, s2 = make_switcher(m1), make_switcher(m2)
+    routes = make_routes(np.array([[0, 1], [2, 3]], np.int32),
+                         np.array([[0.7, 0.3], [0.6, 0.4]], np.float32))
+    p = lambda t: Bnd.Switcher.route_ptr(routes, t)
+    s1.switch(p(0), p(1), stream())
+    s2.switch_layers(0, 1, p(0), p(1), stream())
+    s2.switch_layers(1, 0, p(0), p(1), stream())
+    s2.switch_layers(1, 2, p(0), p(1), stream())
+    torch.cuda.synchronize()
+    for a, b in zip(m1.W, m2.W):
+        assert np.array_equal(bits(a), bits(b))
+    with pytest.raises(Bnd.AdafuseError):
+        s2.switch_layers(2, 2, p(0), p(1), stream())
+
+
+@pytest.mark.parametrize("bad", ["index_high", "index_low", "gate_nan", "gate_inf"])
+def test_bad_route_sets_status_and_writes_nothing(bad):
+    model = _small_model(seed=5)
+    sw = make_switcher(model)
+    W0 = [bits(w) for w in model.W]
+    idx = np.array([[0, 1], [2, 3]], np.int32)
+    gate = np.array([[0.6, 0.4], [0.5, 0.5]], np.float32)
+    if bad == "index_high":
+        idx[1, 1] = 4
+    elif bad == "index_low":
+        idx[1, 0] = -2
+    elif bad == "gate_nan":
+        gate[1, 0] = np.nan
+    else:
+        gate[1, 1] = np.inf
+    routes = make_routes(idx, gate)
+    sw.switch(Bnd.Switcher.route_ptr(routes, 0), Bnd.Switcher.route_ptr(routes, 1), stream())
+    st = sw.status(stream())
+    want = Bnd.ADAFUSE_STATUS_BAD_EXPERT if bad.startswith("index") else Bnd.ADAFUSE_STATUS_BAD_GATE
+    assert st == want
+    assert sw.status(stream()) == 0          # reading clears it
+    for w, w0 in zip(model.W, W0):
+        assert np.array_equal(bits(w), w0)
+
+
+def test_gate_on_empty_slot_is_ignored():
+    model = _small_model(seed=6)
+    sw = make_switcher(model)
+    routes = make_routes(np.array([[1, -1]], np.int32), np.array([[1.0, np.nan]], np.float32))
+    W0 = [bits(w) for w in model.W]
+    sw.switch(None, Bnd.Switcher.route_ptr(routes, 0), stream())
+    assert sw.status(stream()) == 0
+    A_h, B_h = host_ab(model)
+    for i, w in enumerate(model.W):
+        want = oracle.switch(W0[i], A_h[i], B_h[i], model.cfg.scale, None,
+                             (np.array([1, -1], np.int32), np.array([1.0, 0.0], np.float32)))
+        assert ulp_dist(bits(w), want).max() <= MAX_ULP
+
+
+# --------------------------------------------------------------------------
+# full Llama-shaped sizes, the launch the benchmark times, sampled rows
+
+def _sample_rows(cfg, full_layers=()):
+    nt = len(cfg.targets)
+
+    def rows_of(i, out):
+        layer = i // nt
+        if layer in full_layers:
+            return np.arange(out, dtype=np.int64)
+        off = (layer * 7 + (i % nt) * 13) % 97
+        return np.arange(off, out, 97, dtype=np.int64)
+    return rows_of
+
+
+def _full_size_case(name, n_switches, full_first=True):
+    cfg = wl.CONFIGS[name]
+    torch.cuda.empty_cache()
+    model = wl.make_model(cfg, device="cuda")
+    sw = make_switcher(model)
+    A_h, B_h = host_ab(model)
+    if cfg.route_mode == "router":
+        h = wl.make_hidden(cfg, T=n_switches, device="cuda")
+        routes, routes_np, amb = check_pregate(sw, h, model.Wr, cfg.n_experts)
+        assert len(amb) <= 1
+    else:
+        idx, gate = wl.synth_routes(cfg, T=n_switches)
+        routes = make_routes(idx, gate)
+        routes_np = routes_to_np(routes)
+    L = cfg.n_layers
+    if full_first:
+        lockstep(sw, model, routes_np, routes, [(None, 0)],
+                 _sample_rows(cfg, full_layers=(0, L - 1)), A_h, B_h)
+    steps = [(t - 1, t) for t in range(1, n_switches)]
+    lockstep(sw, model, routes_np, routes, steps, _sample_rows(cfg), A_h, B_h)
+    sw.close()
+    del model
+    torch.cuda.empty_cache()
+
+
+def test_llama2_7b_shape_sampled():
+    _full_size_case("7b", 3)
+
+
+def test_llama2_7b_r64_shape_sampled():
+    _full_size_case("7b-r64", 3, full_first=False)
+
+
+def test_llama2_13b_shape_sampled():
+    _full_size_case("13b", 2, full_first=False)
+
+
+def test_llama3_8b_gqa_shape_sampled():
+    _full_size_case("l3-8b", 3, full_first=False)

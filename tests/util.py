@@ -1,0 +1,66 @@
+"""Test helpers: bit-pattern conversions and comparisons (no method arithmetic)."""
+import numpy as np
+import torch
+
+
+def bits(t: torch.Tensor) -> np.ndarray:
+    """bf16 tensor (any device) -> uint16 numpy bit patterns."""
+    return t.detach().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def from_bits(b: np.ndarray, device="cpu") -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).view(torch.bfloat16).to(device)
+
+
+def ordered(u: np.ndarray) -> np.ndarray:
+    u = u.astype(np.int32)
+    return np.where(u & 0x8000, -(u & 0x7FFF), u)
+
+
+def ulp_dist(a: np.ndarray, b: np.ndarray) -> np.ndarray:
+    """Distance in bf16 steps between bit patterns (+0 == -0)."""
+    return np.abs(ordered(a) - ordered(b))
+
+
+def route_tuple(routes_np: np.ndarray, t: int):
+    """Row t of an int32 [T, 4] route buffer -> (idx[2], gate[2]) for the oracle."""
+    row = routes_np[t]
+    return (row[:2].astype(np.int32), row[2:].view(np.float32).copy())
+
+
+def routes_to_np(routes: torch.Tensor) -> np.ndarray:
+    return routes.cpu().numpy().view(np.int32).reshape(-1, 4)
+
+
+def make_routes(idx: np.ndarray, gate: np.ndarray, device="cuda") -> torch.Tensor:
+    """idx [T,2] int32 + gate [T,2] fp32 -> device int32 [T, 4] route buffer."""
+    T = idx.shape[0]
+    buf = np.zeros((T, 4), dtype=np.int32)
+    buf[:, :2] = idx
+    buf[:, 2:] = np.ascontiguousarray(gate, dtype=np.float32).view(np.int32)
+    return torch.from_numpy(buf).to(device)
+
+
+def pregate_consistent(idx_gpu, idx_ref, z, h, Wr):
+    """Accept a top-2 choice that differs from the fp64 oracle only where the
+    fp32 rounding bound 2*d*2^-24*sum|h_i Wr_ie| makes the order ambiguous.
+    Returns (number of exact matches, list of ambiguous token indices)."""
+    T, d = h.shape
+    bound = 2.0 * d * 2.0 ** -24 * (np.abs(h.astype(np.float64)) @ np.abs(Wr.astype(np.float64)))
+    exact, ambiguous = 0, []
+    for t in range(T):
+        a, b = int(idx_gpu[t, 0]), int(idx_gpu[t, 1])
+        if a == idx_ref[t, 0] and b == idx_ref[t, 1]:
+            exact += 1
+            continue
+        E = z.shape[1]
+
+        def can_precede(x, y):
+            return z[t, x] + bound[t, x] >= z[t, y] - bound[t, y]
+        ok = 0 <= a < E and (b == -1 or 0 <= b < E) and a != b
+        ok = ok and all(can_precede(a, e) for e in range(E) if e != a)
+        if b >= 0:
+            ok = ok and all(can_precede(b, e) for e in range(E) if e not in (a, b))
+        assert ok, f"token {t}: gpu picked {(a, b)}, oracle {tuple(idx_ref[t])}, z={z[t]}"
+        ambiguous.append(t)
+    return exact, ambiguous

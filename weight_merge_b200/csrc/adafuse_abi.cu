@@ -1,0 +1,320 @@
+// adafuse_abi.cu -- C ABI of the adapter switch: context, segment table,
+// argument checks and kernel launches.  See include/adafuse.h for the
+// contract of each entry point.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "adafuse.h"
+#include "common.cuh"
+#include "pregate.cuh"
+#include "switch_mma.cuh"
+
+using namespace adafuse;
+
+struct adafuse_ctx {
+    int device = 0;
+    int sm_count = 0;
+    int32_t n_layers = 0, n_targets = 0, n_experts = 0, rank = 0;
+    float alpha = 0.f, scale = 0.f;
+    int64_t n_tiles = 0;
+    std::vector<int64_t> layer_tile_begin;  // [n_layers + 1]
+    PairDesc* d_pairs = nullptr;
+    TileEntry* d_tiles = nullptr;
+    int32_t* d_status = nullptr;
+};
+
+namespace {
+
+thread_local char g_last_error[256] = "";
+
+int cuda_fail(cudaError_t e, const char* what) {
+    std::snprintf(g_last_error, sizeof g_last_error, "%s: %s", what, cudaGetErrorString(e));
+    return ADAFUSE_ERR_CUDA;
+}
+
+// Restores the caller's current device on scope exit.
+struct DeviceGuard {
+    int prev = -1;
+    bool ok = false;
+    explicit DeviceGuard(int dev) {
+        if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+        ok = (prev == dev) || cudaSetDevice(dev) == cudaSuccess;
+    }
+    ~DeviceGuard() {
+        if (prev >= 0) cudaSetDevice(prev);
+    }
+};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Shape and pointer checks shared by create and the host-only table query.
+int check_desc(const adafuse_desc* d, bool need_pointers) {
+    if (d == nullptr || d->targets == nullptr) return ADAFUSE_ERR_INVALID_ARG;
+    if (d->n_layers < 1 || d->n_targets < 1) return ADAFUSE_ERR_INVALID_ARG;
+    if (d->n_experts < 1 || d->n_experts > 64) return ADAFUSE_ERR_UNSUPPORTED_SHAPE;
+    if (d->rank < 1 || d->rank > 64) return ADAFUSE_ERR_UNSUPPORTED_SHAPE;
+    if (!std::isfinite(d->alpha)) return ADAFUSE_ERR_INVALID_ARG;
+    const int64_t n = (int64_t)d->n_layers * d->n_targets;
+    if (n > (int64_t)1 << 30) return ADAFUSE_ERR_UNSUPPORTED_SHAPE;
+    for (int64_t i = 0; i < n; ++i) {
+        const adafuse_target& t = d->targets[i];
+        if (t.out <= 0 || t.in <= 0) return ADAFUSE_ERR_INVALID_ARG;
+        if (t.out % 8 != 0 || t.in % 8 != 0) return ADAFUSE_ERR_UNSUPPORTED_SHAPE;
+        // tile indices are packed in 16 bits; element offsets in int32 rows
+        if (ceil_div(t.out, kTile) > 65535 || ceil_div(t.in, kTile) > 65535)
+            return ADAFUSE_ERR_UNSUPPORTED_SHAPE;
+        if (t.out > INT32_MAX || t.in > INT32_MAX) return ADAFUSE_ERR_UNSUPPORTED_SHAPE;
+        if (need_pointers) {
+            if (t.W == nullptr || t.A == nullptr || t.B == nullptr) return ADAFUSE_ERR_INVALID_ARG;
+            if (!aligned16(t.W) || !aligned16(t.A) || !aligned16(t.B)) return ADAFUSE_ERR_INVALID_ARG;
+        }
+    }
+    return ADAFUSE_OK;
+}
+
+// The segment table: every (layer, target) weight cut into 128x128 tiles
+// (the last row / column of tiles may be ragged), layer-major, then target,
+// then row tile, then column tile.  Each W element lies in exactly one tile.
+template <typename Emit>
+int64_t walk_tiles(const adafuse_desc* d, Emit&& emit) {
+    int64_t n = 0;
+    for (int32_t l = 0; l < d->n_layers; ++l)
+        for (int32_t k = 0; k < d->n_targets; ++k) {
+            const adafuse_target& t = d->targets[(int64_t)l * d->n_targets + k];
+            const int64_t rt = ceil_div(t.out, kTile), ct = ceil_div(t.in, kTile);
+            for (int64_t i = 0; i < rt; ++i)
+                for (int64_t j = 0; j < ct; ++j) emit(l, k, i, j, n++);
+        }
+    return n;
+}
+
+int kp_class(int r) { return r <= 8 ? 8 : r <= 16 ? 16 : r <= 32 ? 32 : 64; }
+
+}  // namespace
+
+extern "C" {
+
+const char* adafuse_last_error(void) { return g_last_error; }
+
+const char* adafuse_strerror(int code) {
+    switch (code) {
+        case ADAFUSE_OK: return "ok";
+        case ADAFUSE_ERR_INVALID_ARG: return "invalid argument";
+        case ADAFUSE_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+        case ADAFUSE_ERR_CUDA: return "CUDA runtime error";
+        case ADAFUSE_ERR_DEVICE_FAULT: return "device status word set (bad route)";
+        case ADAFUSE_ERR_UNSUPPORTED_DEVICE: return "device is not compute capability 10.0";
+        case ADAFUSE_ERR_OUT_OF_MEMORY: return "out of memory";
+        default: return "unknown error";
+    }
+}
+
+int adafuse_tile_size(void) { return kTile; }
+
+int adafuse_segment_table(const adafuse_desc* desc, int32_t* entries, int64_t capacity,
+                          int64_t* count) {
+    if (count == nullptr) return ADAFUSE_ERR_INVALID_ARG;
+    const int rc = check_desc(desc, false);
+    if (rc != ADAFUSE_OK) return rc;
+    const int64_t n = walk_tiles(desc, [](int, int, int64_t, int64_t, int64_t) {});
+    *count = n;
+    if (entries == nullptr) return ADAFUSE_OK;
+    if (capacity < n) return ADAFUSE_ERR_INVALID_ARG;
+    walk_tiles(desc, [&](int l, int k, int64_t i, int64_t j, int64_t q) {
+        entries[4 * q + 0] = l;
+        entries[4 * q + 1] = k;
+        entries[4 * q + 2] = (int32_t)(i * kTile);
+        entries[4 * q + 3] = (int32_t)(j * kTile);
+    });
+    return ADAFUSE_OK;
+}
+
+int adafuse_create(adafuse_ctx** out, const adafuse_desc* desc, int device) {
+    if (out == nullptr) return ADAFUSE_ERR_INVALID_ARG;
+    *out = nullptr;
+    int rc = check_desc(desc, true);
+    if (rc != ADAFUSE_OK) return rc;
+
+    int ndev = 0;
+    cudaError_t e = cudaGetDeviceCount(&ndev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDeviceCount");
+    if (device < 0 || device >= ndev) return ADAFUSE_ERR_INVALID_ARG;
+    DeviceGuard guard(device);
+    if (!guard.ok) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
+    cudaDeviceProp prop;
+    e = cudaGetDeviceProperties(&prop, device);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDeviceProperties");
+    if (prop.major != 10 || prop.minor != 0) return ADAFUSE_ERR_UNSUPPORTED_DEVICE;
+
+    adafuse_ctx* c = new (std::nothrow) adafuse_ctx();
+    if (c == nullptr) return ADAFUSE_ERR_OUT_OF_MEMORY;
+    c->device = device;
+    c->sm_count = prop.multiProcessorCount;
+    c->n_layers = desc->n_layers;
+    c->n_targets = desc->n_targets;
+    c->n_experts = desc->n_experts;
+    c->rank = desc->rank;
+    c->alpha = desc->alpha;
+    c->scale = desc->alpha / (float)desc->rank;
+
+    const int64_t npairs = (int64_t)desc->n_layers * desc->n_targets;
+    std::vector<PairDesc> pairs((size_t)npairs);
+    for (int64_t i = 0; i < npairs; ++i) {
+        const adafuse_target& t = desc->targets[i];
+        pairs[i].W = static_cast<uint16_t*>(t.W);
+        pairs[i].A = static_cast<const uint16_t*>(t.A);
+        pairs[i].B = static_cast<const uint16_t*>(t.B);
+        pairs[i].out = (int32_t)t.out;
+        pairs[i].in = (int32_t)t.in;
+        pairs[i].layer = (int32_t)(i / desc->n_targets);
+        pairs[i].target = (int32_t)(i % desc->n_targets);
+    }
+    std::vector<TileEntry> tiles;
+    c->layer_tile_begin.assign((size_t)desc->n_layers + 1, 0);
+    try {
+        tiles.reserve((size_t)walk_tiles(desc, [](int, int, int64_t, int64_t, int64_t) {}));
+        walk_tiles(desc, [&](int l, int k, int64_t i, int64_t j, int64_t) {
+            TileEntry te;
+            te.x = (uint32_t)((int64_t)l * desc->n_targets + k);
+            te.y = (uint32_t)((i << 16) | j);
+            tiles.push_back(te);
+            c->layer_tile_begin[(size_t)l + 1] = (int64_t)tiles.size();
+        });
+    } catch (...) {
+        delete c;
+        return ADAFUSE_ERR_OUT_OF_MEMORY;
+    }
+    c->n_tiles = (int64_t)tiles.size();
+
+    auto fail = [&](cudaError_t err, const char* what) {
+        cudaFree(c->d_pairs);
+        cudaFree(c->d_tiles);
+        cudaFree(c->d_status);
+        delete c;
+        return err == cudaErrorMemoryAllocation ? ADAFUSE_ERR_OUT_OF_MEMORY : cuda_fail(err, what);
+    };
+    if ((e = cudaMalloc(&c->d_pairs, sizeof(PairDesc) * pairs.size())) != cudaSuccess)
+        return fail(e, "cudaMalloc(pairs)");
+    if ((e = cudaMalloc(&c->d_tiles, sizeof(TileEntry) * tiles.size())) != cudaSuccess)
+        return fail(e, "cudaMalloc(tiles)");
+    if ((e = cudaMalloc(&c->d_status, sizeof(int32_t))) != cudaSuccess)
+        return fail(e, "cudaMalloc(status)");
+    if ((e = cudaMemcpy(c->d_pairs, pairs.data(), sizeof(PairDesc) * pairs.size(),
+                        cudaMemcpyHostToDevice)) != cudaSuccess)
+        return fail(e, "cudaMemcpy(pairs)");
+    if ((e = cudaMemcpy(c->d_tiles, tiles.data(), sizeof(TileEntry) * tiles.size(),
+                        cudaMemcpyHostToDevice)) != cudaSuccess)
+        return fail(e, "cudaMemcpy(tiles)");
+    if ((e = cudaMemset(c->d_status, 0, sizeof(int32_t))) != cudaSuccess)
+        return fail(e, "cudaMemset(status)");
+    *out = c;
+    return ADAFUSE_OK;
+}
+
+int adafuse_destroy(adafuse_ctx* ctx) {
+    if (ctx == nullptr) return ADAFUSE_OK;
+    DeviceGuard guard(ctx->device);
+    cudaFree(ctx->d_pairs);
+    cudaFree(ctx->d_tiles);
+    cudaFree(ctx->d_status);
+    delete ctx;
+    return ADAFUSE_OK;
+}
+
+int adafuse_pregate(adafuse_ctx* ctx, const float* h, int64_t T, int64_t d, const float* Wr,
+                    adafuse_route* route, void* stream) {
+    if (ctx == nullptr || T < 0 || d < 1 || (d & 3) != 0) return ADAFUSE_ERR_INVALID_ARG;
+    if (T == 0) return ADAFUSE_OK;
+    if (h == nullptr || Wr == nullptr || route == nullptr) return ADAFUSE_ERR_INVALID_ARG;
+    if (!aligned16(h) || !aligned16(route) || (reinterpret_cast<uintptr_t>(Wr) & 3u))
+        return ADAFUSE_ERR_INVALID_ARG;
+    DeviceGuard guard(ctx->device);
+    if (!guard.ok) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int E = ctx->n_experts;
+    if (E <= 8) {
+        constexpr int TPB = 8;
+        pregate_kernel<8, TPB><<<(unsigned)ceil_div(T, TPB), kPregateThreads, 0, s>>>(h, T, d, Wr, E, route);
+    } else if (E <= 16) {
+        constexpr int TPB = 4;
+        pregate_kernel<16, TPB><<<(unsigned)ceil_div(T, TPB), kPregateThreads, 0, s>>>(h, T, d, Wr, E, route);
+    } else if (E <= 32) {
+        constexpr int TPB = 2;
+        pregate_kernel<32, TPB><<<(unsigned)ceil_div(T, TPB), kPregateThreads, 0, s>>>(h, T, d, Wr, E, route);
+    } else {
+        constexpr int TPB = 1;
+        pregate_kernel<64, TPB><<<(unsigned)ceil_div(T, TPB), kPregateThreads, 0, s>>>(h, T, d, Wr, E, route);
+    }
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? ADAFUSE_OK : cuda_fail(e, "pregate launch");
+}
+
+int adafuse_switch_batch_layers(adafuse_ctx* ctx, int32_t layer_begin, int32_t n_layers,
+                                const adafuse_route* prev, const adafuse_route* cur,
+                                void* stream) {
+    if (ctx == nullptr || n_layers < 0 || layer_begin < 0) return ADAFUSE_ERR_INVALID_ARG;
+    if ((int64_t)layer_begin + n_layers > ctx->n_layers) return ADAFUSE_ERR_INVALID_ARG;
+    if (!aligned16(prev) || !aligned16(cur)) return ADAFUSE_ERR_INVALID_ARG;
+    if (n_layers == 0) return ADAFUSE_OK;
+    const int64_t t0 = ctx->layer_tile_begin[(size_t)layer_begin];
+    const int64_t t1 = ctx->layer_tile_begin[(size_t)layer_begin + n_layers];
+    if (t1 <= t0) return ADAFUSE_OK;
+    DeviceGuard guard(ctx->device);
+    if (!guard.ok) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t want = (int64_t)ctx->sm_count * 2;
+    const unsigned grid = (unsigned)(t1 - t0 < want ? t1 - t0 : want);
+    const int E = ctx->n_experts, r = ctx->rank;
+    const float sc = ctx->scale;
+    switch (kp_class(r)) {
+        case 8:
+            switch_mma_kernel<8><<<grid, kSwitchThreads, 0, s>>>(ctx->d_pairs, ctx->d_tiles, t0, t1,
+                                                                 prev, cur, E, r, sc, ctx->d_status);
+            break;
+        case 16:
+            switch_mma_kernel<16><<<grid, kSwitchThreads, 0, s>>>(ctx->d_pairs, ctx->d_tiles, t0, t1,
+                                                                  prev, cur, E, r, sc, ctx->d_status);
+            break;
+        case 32:
+            switch_mma_kernel<32><<<grid, kSwitchThreads, 0, s>>>(ctx->d_pairs, ctx->d_tiles, t0, t1,
+                                                                  prev, cur, E, r, sc, ctx->d_status);
+            break;
+        default:
+            switch_mma_kernel<64><<<grid, kSwitchThreads, 0, s>>>(ctx->d_pairs, ctx->d_tiles, t0, t1,
+                                                                  prev, cur, E, r, sc, ctx->d_status);
+            break;
+    }
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? ADAFUSE_OK : cuda_fail(e, "switch launch");
+}
+
+int adafuse_switch(adafuse_ctx* ctx, const adafuse_route* prev, const adafuse_route* cur,
+                   void* stream) {
+    if (ctx == nullptr) return ADAFUSE_ERR_INVALID_ARG;
+    return adafuse_switch_batch_layers(ctx, 0, ctx->n_layers, prev, cur, stream);
+}
+
+int adafuse_get_device_status(adafuse_ctx* ctx, void* stream, int32_t* status) {
+    if (ctx == nullptr || status == nullptr) return ADAFUSE_ERR_INVALID_ARG;
+    DeviceGuard guard(ctx->device);
+    if (!guard.ok) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t v = 0;
+    cudaError_t e = cudaMemcpyAsync(&v, ctx->d_status, sizeof v, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ctx->d_status, 0, sizeof v, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "device status read");
+    *status = v;
+    return v == 0 ? ADAFUSE_OK : ADAFUSE_ERR_DEVICE_FAULT;
+}
+
+}  // extern "C"
