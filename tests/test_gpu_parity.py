@@ -17,8 +17,8 @@ import oracle
 from weight_merge_b200 import binding as Bnd
 from weight_merge_b200 import workloads as wl
 
-from .util import (bits, make_routes, pregate_consistent, route_tuple, routes_to_np,
-                   ulp_dist)
+from .util import (bits, check_switch_rows, make_routes, pregate_consistent, route_tuple,
+                   routes_to_np, ulp_dist)
 
 pytestmark = pytest.mark.gpu
 
@@ -66,10 +66,11 @@ def check_pregate(sw, h, Wr, E):
 
 def lockstep(sw, model, routes_np, routes_dev, steps, rows_of, A_h, B_h):
     """Run switches (prev_t, cur_t) -- None = no route -- and compare the rows
-    rows_of(pair_index, out) of every weight with the oracle after each."""
+    rows_of(pair_index, out) of every weight with the oracle after each.
+    Returns (worst step distance, cancellation-clause elements, elements checked)."""
     cfg = model.cfg
     nt = len(cfg.targets)
-    worst = 0
+    worst = ncancel = nchecked = 0
     for (p, c) in steps:
         sel = [rows_of(i, w.shape[0]) for i, w in enumerate(model.W)]
         before = [bits(w[torch.as_tensor(r, device="cuda")]) for w, r in zip(model.W, sel)]
@@ -81,17 +82,17 @@ def lockstep(sw, model, routes_np, routes_dev, steps, rows_of, A_h, B_h):
         cur = route_tuple(routes_np, c) if c is not None else None
         for i, w in enumerate(model.W):
             after = bits(w[torch.as_tensor(sel[i], device="cuda")])
-            want = oracle.switch_rows(before[i], sel[i], w.shape[0], A_h[i], B_h[i], cfg.scale,
-                                      prev, cur)
-            d = ulp_dist(after, want)
-            if d.max() > MAX_ULP:
-                bad = np.argwhere(d > MAX_ULP)[0]
-                raise AssertionError(
-                    f"switch {(p, c)} layer {i // nt} target {cfg.targets[i % nt].name} "
-                    f"row {sel[i][bad[0]]} col {bad[1]}: gpu {after[tuple(bad)]:#06x} "
-                    f"oracle {want[tuple(bad)]:#06x} ({d.max()} steps)")
-            worst = max(worst, int(d.max()))
-    return worst
+            try:
+                wd, nc = check_switch_rows(after, before[i], sel[i], w.shape[0], A_h[i], B_h[i],
+                                           cfg.scale, prev, cur, MAX_ULP)
+            except AssertionError as ex:
+                raise AssertionError(f"switch {(p, c)} layer {i // nt} target "
+                                     f"{cfg.targets[i % nt].name}: {ex}") from None
+            worst, ncancel = max(worst, wd), ncancel + nc
+            nchecked += after.size
+    # the cancellation clause is for rare elements only
+    assert ncancel <= max(2, nchecked * 1e-5), (ncancel, nchecked)
+    return worst, ncancel, nchecked
 
 
 def all_rows(i, out):
@@ -265,9 +266,9 @@ def test_gate_on_empty_slot_is_ignored():
     assert sw.status(stream()) == 0
     A_h, B_h = host_ab(model)
     for i, w in enumerate(model.W):
-        want = oracle.switch(W0[i], A_h[i], B_h[i], model.cfg.scale, None,
-                             (np.array([1, -1], np.int32), np.array([1.0, 0.0], np.float32)))
-        assert ulp_dist(bits(w), want).max() <= MAX_ULP
+        rows = np.arange(w.shape[0], dtype=np.int64)
+        check_switch_rows(bits(w), W0[i], rows, w.shape[0], A_h[i], B_h[i], model.cfg.scale,
+                          None, (np.array([1, -1], np.int32), np.array([1.0, 0.0], np.float32)))
 
 
 # --------------------------------------------------------------------------

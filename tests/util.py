@@ -64,3 +64,58 @@ def pregate_consistent(idx_gpu, idx_ref, z, h, Wr):
         assert ok, f"token {t}: gpu picked {(a, b)}, oracle {tuple(idx_ref[t])}, z={z[t]}"
         ambiguous.append(t)
     return exact, ambiguous
+
+
+def bf16_to_f64(b: np.ndarray) -> np.ndarray:
+    return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def bf16_step(b: np.ndarray) -> np.ndarray:
+    """Spacing of bf16 values at the given bit patterns (2^-133 when subnormal)."""
+    e = (b.astype(np.int32) >> 7) & 0xFF
+    return np.ldexp(1.0, np.where(e == 0, -133, e - 127 - 7))
+
+
+def fp32_accum_gamma(rank: int) -> float:
+    """Relative error bound of the fp32 path: rank products summed per expert,
+    up to four expert terms and W combined, the coefficient rounded once."""
+    return (rank + 8) * 2.0 ** -24
+
+
+def check_switch_rows(after, before, rows, out, A, B, s, prev, cur, max_ulp=1):
+    """Compare GPU rows with the oracle.
+
+    Pass per element if it is within `max_ulp` bf16 steps of the oracle's
+    bf16_rne(W + dW), or -- where the result cancels far below the terms it
+    is formed from -- within half a step plus the fp32 accumulation bound
+    gamma * (|W| + s * sum_e g_e sum_k |B_ek| |A_kj|) of the exact value.
+    Returns (worst step distance, number of elements that needed the
+    cancellation clause)."""
+    import oracle
+    want, exact = oracle.switch_rows(before, rows, out, A, B, s, prev, cur, exact=True)
+    d = ulp_dist(after, want)
+    bad = d > max_ulp
+    if not bad.any():
+        return int(d.max()) if d.size else 0, 0
+    brows = np.unique(np.nonzero(bad)[0])
+    M = np.abs(bf16_to_f64(before[brows]))
+    Af, Bf = np.abs(bf16_to_f64(A)), np.abs(bf16_to_f64(B))
+    for rt in (prev, cur):
+        if rt is None:
+            continue
+        for e, g in zip(rt[0], rt[1]):
+            if e < 0:
+                continue
+            M += s * abs(float(g)) * (Bf[e][rows[brows]] @ Af[e])
+    r = A.shape[1]
+    gpu = bf16_to_f64(after[brows])
+    tol = 0.5 * bf16_step(after[brows]) + fp32_accum_gamma(r) * M
+    sub_bad = bad[brows]
+    err = np.abs(gpu - exact[brows])
+    ok = err <= tol
+    if not np.all(ok[sub_bad]):
+        i, j = np.argwhere(sub_bad & ~ok)[0]
+        raise AssertionError(
+            f"row {rows[brows[i]]} col {j}: gpu {gpu[i, j]!r} exact {exact[brows[i], j]!r} "
+            f"err {err[i, j]:.3e} > tol {tol[i, j]:.3e} ({d[brows[i], j]} steps)")
+    return int(d[~bad].max()) if (~bad).any() else 0, int(bad.sum())
