@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--config", default="7b")
     ap.add_argument("--layers", type=int, default=None,
                     help="override the layer count (small cases for ncu captures)")
+    ap.add_argument("--kernel", choices=["auto", "mma", "tc"], default="auto",
+                    help="switch kernel: tensor-core (tc), mma.sync (mma), or auto")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--traffic-gb", type=float, default=None,
@@ -232,6 +234,10 @@ def run_ours(args):
     model = wl.make_model(cfg, device="cuda")
     sw = B.Switcher(model.W, model.A, model.B, cfg.n_layers, len(cfg.targets), cfg.n_experts,
                     cfg.rank, cfg.alpha, device=dev, names=[t.name for t in cfg.targets])
+    sw.set_kernel({"auto": B.ADAFUSE_KERNEL_AUTO, "mma": B.ADAFUSE_KERNEL_MMA_SYNC,
+                   "tc": B.ADAFUSE_KERNEL_TCGEN05}[args.kernel])
+    kernel_name = {B.ADAFUSE_KERNEL_MMA_SYNC: "switch_mma_kernel",
+                   B.ADAFUSE_KERNEL_TCGEN05: "switch_tc_kernel"}[sw.kernel]
     T = cfg.n_tokens
     h = wl.make_hidden(cfg, T=T, device="cuda")
     routes = torch.zeros((T, 4), dtype=torch.int32, device="cuda")
@@ -373,7 +379,7 @@ def run_ours(args):
                          "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "peak_kind": peak_kind,
                          "traffic": (round(args.traffic_gb * 1e9) if args.traffic_gb else None),
-                         "kernel": "switch_mma_kernel"},
+                         "kernel": kernel_name},
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": 2 * args.steps,

@@ -78,6 +78,13 @@ extern "C" {
 /* ---- device status word bits (adafuse_get_device_status) ---------------- */
 #define ADAFUSE_STATUS_BAD_EXPERT   0x1   /* a route held an index outside [-1, E) */
 #define ADAFUSE_STATUS_BAD_GATE     0x2   /* a route held a non-finite gate on a used slot */
+#define ADAFUSE_STATUS_TIMEOUT      0x4   /* a bounded wait inside the switch kernel gave up
+                                             (the switch is then incomplete) */
+
+/* ---- switch kernel variants (adafuse_set_switch_kernel) ------------------ */
+#define ADAFUSE_KERNEL_AUTO      0  /* tensor-core kernel when the rank allows it, else mma.sync */
+#define ADAFUSE_KERNEL_MMA_SYNC  1  /* register-streaming kernel, any rank in [1, 64] */
+#define ADAFUSE_KERNEL_TCGEN05   2  /* TMA + tcgen05/TMEM kernel, rank a multiple of 8 */
 
 /* One token's routing decision: the two chosen experts and their gates.
  * idx[j] == -1 marks an empty slot (its gate is ignored).  adafuse_pregate
@@ -163,6 +170,16 @@ ADAFUSE_API int adafuse_switch(adafuse_ctx* ctx, const adafuse_route* prev,
 ADAFUSE_API int adafuse_switch_batch_layers(adafuse_ctx* ctx, int32_t layer_begin,
                                 int32_t n_layers, const adafuse_route* prev,
                                 const adafuse_route* cur, void* stream);
+
+/* Choose the kernel adafuse_switch launches for this context (default
+ * ADAFUSE_KERNEL_AUTO).  Both compute the same update to within the
+ * documented rounding; ADAFUSE_KERNEL_TCGEN05 needs rank % 8 == 0 and
+ * returns UNSUPPORTED_SHAPE otherwise.  Host-only, no device work. */
+ADAFUSE_API int adafuse_set_switch_kernel(adafuse_ctx* ctx, int kernel);
+
+/* The kernel adafuse_switch will launch (ADAFUSE_KERNEL_MMA_SYNC or
+ * ADAFUSE_KERNEL_TCGEN05), or a negative code. */
+ADAFUSE_API int adafuse_get_switch_kernel(adafuse_ctx* ctx);
 
 /* Synchronise `stream`, read the device status word into *status, then
  * clear it.  Returns ADAFUSE_ERR_DEVICE_FAULT when the word was non-zero,

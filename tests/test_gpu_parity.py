@@ -38,11 +38,22 @@ def stream():
     return torch.cuda.current_stream().cuda_stream
 
 
-def make_switcher(model: wl.Model) -> Bnd.Switcher:
+MMA, TC = Bnd.ADAFUSE_KERNEL_MMA_SYNC, Bnd.ADAFUSE_KERNEL_TCGEN05
+
+
+def make_switcher(model: wl.Model, kernel: int = Bnd.ADAFUSE_KERNEL_AUTO) -> Bnd.Switcher:
     c = model.cfg
-    return Bnd.Switcher(model.W, model.A, model.B, c.n_layers, len(c.targets), c.n_experts,
-                        c.rank, c.alpha, device=torch.cuda.current_device(),
-                        names=[t.name for t in c.targets])
+    sw = Bnd.Switcher(model.W, model.A, model.B, c.n_layers, len(c.targets), c.n_experts,
+                      c.rank, c.alpha, device=torch.cuda.current_device(),
+                      names=[t.name for t in c.targets])
+    sw.set_kernel(kernel)
+    if kernel != Bnd.ADAFUSE_KERNEL_AUTO:
+        assert sw.kernel == kernel
+    return sw
+
+
+def kernels_for(rank):
+    return [MMA, TC] if rank % 8 == 0 else [MMA]
 
 
 def host_ab(model):
@@ -151,13 +162,15 @@ def test_tiny_sequence_lockstep_all_elements():
 RAGGED = [("a", 200, 136), ("b", 8, 8), ("c", 264, 392), ("d", 128, 256), ("e", 136, 8)]
 
 
-@pytest.mark.parametrize("E,r", [(1, 1), (3, 3), (4, 4), (5, 8), (16, 12), (4, 16), (6, 24),
-                                 (3, 32), (4, 40), (5, 64)])
-def test_ragged_shapes_every_rank_class(E, r):
+RANKS = [(1, 1), (3, 3), (4, 4), (5, 8), (16, 12), (4, 16), (6, 24), (3, 32), (4, 40), (5, 64)]
+
+
+@pytest.mark.parametrize("E,r,kernel", [(E, r, k) for (E, r) in RANKS for k in kernels_for(r)])
+def test_ragged_shapes_every_rank_class(E, r, kernel):
     cfg = wl.custom("ragged", 2, RAGGED, n_experts=E, rank=r, alpha=2.0 * r, n_tokens=6,
                     d=136)
     model = wl.make_model(cfg, device="cuda", seed=1000 + 7 * r + E)
-    sw = make_switcher(model)
+    sw = make_switcher(model, kernel)
     rng = np.random.default_rng(r * 31 + E)
     T = 6
     idx = rng.integers(0, E, size=(T, 2)).astype(np.int32)
@@ -180,9 +193,10 @@ def _small_model(seed=3, E=4, r=8):
     return wl.make_model(cfg, device="cuda", seed=seed)
 
 
-def test_identity_switches_leave_w_bit_identical():
+@pytest.mark.parametrize("kernel", [MMA, TC])
+def test_identity_switches_leave_w_bit_identical(kernel):
     model = _small_model()
-    sw = make_switcher(model)
+    sw = make_switcher(model, kernel)
     W0 = [bits(w) for w in model.W]
     idx = np.array([[1, 2], [2, 1], [0, 3]], dtype=np.int32)
     gate = np.array([[0.8, 0.2], [0.2, 0.8], [0.0, 0.0]], dtype=np.float32)
@@ -196,9 +210,10 @@ def test_identity_switches_leave_w_bit_identical():
         assert np.array_equal(bits(w), w0)
 
 
-def test_merge_then_unmerge_restores_within_rounding():
+@pytest.mark.parametrize("kernel", [MMA, TC])
+def test_merge_then_unmerge_restores_within_rounding(kernel):
     model = _small_model(seed=4)
-    sw = make_switcher(model)
+    sw = make_switcher(model, kernel)
     W0 = [bits(w) for w in model.W]
     routes = make_routes(np.array([[0, 3]], np.int32), np.array([[0.55, 0.45]], np.float32))
     sw.switch(None, Bnd.Switcher.route_ptr(routes, 0), stream())
@@ -215,9 +230,10 @@ def test_merge_then_unmerge_restores_within_rounding():
         assert np.all(np.abs(f(w2) - f(w0)) <= 0.5 * e(w1) + 0.5 * e(w2) + 1e-30)
 
 
-def test_layer_ranges_equal_one_full_switch():
+@pytest.mark.parametrize("kernel", [MMA, TC])
+def test_layer_ranges_equal_one_full_switch(kernel):
     m1, m2 = _small_model(seed=9), _small_model(seed=9)
-    s1, s2 = make_switcher(m1), make_switcher(m2)
+    s1, s2 = make_switcher(m1, kernel), make_switcher(m2, kernel)
     routes = make_routes(np.array([[0, 1], [2, 3]], np.int32),
                          np.array([[0.7, 0.3], [0.6, 0.4]], np.float32))
     p = lambda t: Bnd.Switcher.route_ptr(routes, t)
@@ -232,10 +248,11 @@ def test_layer_ranges_equal_one_full_switch():
         s2.switch_layers(2, 2, p(0), p(1), stream())
 
 
+@pytest.mark.parametrize("kernel", [MMA, TC])
 @pytest.mark.parametrize("bad", ["index_high", "index_low", "gate_nan", "gate_inf"])
-def test_bad_route_sets_status_and_writes_nothing(bad):
+def test_bad_route_sets_status_and_writes_nothing(bad, kernel):
     model = _small_model(seed=5)
-    sw = make_switcher(model)
+    sw = make_switcher(model, kernel)
     W0 = [bits(w) for w in model.W]
     idx = np.array([[0, 1], [2, 3]], np.int32)
     gate = np.array([[0.6, 0.4], [0.5, 0.5]], np.float32)
@@ -257,9 +274,10 @@ def test_bad_route_sets_status_and_writes_nothing(bad):
         assert np.array_equal(bits(w), w0)
 
 
-def test_gate_on_empty_slot_is_ignored():
+@pytest.mark.parametrize("kernel", [MMA, TC])
+def test_gate_on_empty_slot_is_ignored(kernel):
     model = _small_model(seed=6)
-    sw = make_switcher(model)
+    sw = make_switcher(model, kernel)
     routes = make_routes(np.array([[1, -1]], np.int32), np.array([[1.0, np.nan]], np.float32))
     W0 = [bits(w) for w in model.W]
     sw.switch(None, Bnd.Switcher.route_ptr(routes, 0), stream())
@@ -286,11 +304,12 @@ def _sample_rows(cfg, full_layers=()):
     return rows_of
 
 
-def _full_size_case(name, n_switches, full_first=True):
+def _full_size_case(name, n_switches, full_first=True, kernel=Bnd.ADAFUSE_KERNEL_AUTO):
     cfg = wl.CONFIGS[name]
     torch.cuda.empty_cache()
     model = wl.make_model(cfg, device="cuda")
-    sw = make_switcher(model)
+    sw = make_switcher(model, kernel)
+    assert sw.kernel == TC         # the benchmark's launch configuration
     A_h, B_h = host_ab(model)
     if cfg.route_mode == "router":
         h = wl.make_hidden(cfg, T=n_switches, device="cuda")
@@ -309,6 +328,16 @@ def _full_size_case(name, n_switches, full_first=True):
     sw.close()
     del model
     torch.cuda.empty_cache()
+
+
+def test_auto_picks_tensor_cores_when_rank_allows():
+    for r, want in [(4, MMA), (8, TC), (12, MMA), (16, TC), (64, TC)]:
+        cfg = wl.custom("k", 1, [("q", 64, 64)], n_experts=2, rank=r, alpha=2.0 * r, n_tokens=1)
+        sw = make_switcher(wl.make_model(cfg, device="cuda"))
+        assert sw.kernel == want
+        if want == MMA:
+            with pytest.raises(Bnd.AdafuseError):
+                sw.set_kernel(TC)
 
 
 def test_llama2_7b_shape_sampled():

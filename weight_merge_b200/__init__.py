@@ -9,8 +9,10 @@ importing the binding fails loudly when the compiled library is missing.
 from .binding import (  # noqa: F401
     ADAFUSE_OK, ADAFUSE_ERR_INVALID_ARG, ADAFUSE_ERR_UNSUPPORTED_SHAPE, ADAFUSE_ERR_CUDA,
     ADAFUSE_ERR_DEVICE_FAULT, ADAFUSE_ERR_UNSUPPORTED_DEVICE, ADAFUSE_ERR_OUT_OF_MEMORY,
-    ADAFUSE_STATUS_BAD_EXPERT, ADAFUSE_STATUS_BAD_GATE, AdafuseError, Route, Target, Desc,
+    ADAFUSE_STATUS_BAD_EXPERT, ADAFUSE_STATUS_BAD_GATE, ADAFUSE_STATUS_TIMEOUT,
+    ADAFUSE_KERNEL_AUTO, ADAFUSE_KERNEL_MMA_SYNC, ADAFUSE_KERNEL_TCGEN05, AdafuseError, Route, Target, Desc,
     lib, library_path, adafuse_create, adafuse_destroy, adafuse_pregate, adafuse_switch,
-    adafuse_switch_batch_layers, adafuse_get_device_status, adafuse_segment_table,
+    adafuse_switch_batch_layers, adafuse_get_device_status, adafuse_set_switch_kernel,
+    adafuse_get_switch_kernel, adafuse_segment_table,
     adafuse_tile_size, adafuse_strerror, adafuse_last_error, Switcher,
 )

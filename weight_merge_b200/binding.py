@@ -23,6 +23,10 @@ ADAFUSE_ERR_UNSUPPORTED_DEVICE = -5
 ADAFUSE_ERR_OUT_OF_MEMORY = -6
 ADAFUSE_STATUS_BAD_EXPERT = 0x1
 ADAFUSE_STATUS_BAD_GATE = 0x2
+ADAFUSE_STATUS_TIMEOUT = 0x4
+ADAFUSE_KERNEL_AUTO = 0
+ADAFUSE_KERNEL_MMA_SYNC = 1
+ADAFUSE_KERNEL_TCGEN05 = 2
 
 
 class AdafuseError(RuntimeError):
@@ -75,6 +79,8 @@ def lib() -> ctypes.CDLL:
         "adafuse_switch": ([P, P, P, P], ctypes.c_int),
         "adafuse_switch_batch_layers": ([P, i32, i32, P, P, P], ctypes.c_int),
         "adafuse_get_device_status": ([P, P, ctypes.POINTER(i32)], ctypes.c_int),
+        "adafuse_set_switch_kernel": ([P, ctypes.c_int], ctypes.c_int),
+        "adafuse_get_switch_kernel": ([P], ctypes.c_int),
         "adafuse_segment_table": ([ctypes.POINTER(Desc), P, i64, ctypes.POINTER(i64)], ctypes.c_int),
         "adafuse_tile_size": ([], ctypes.c_int),
         "adafuse_strerror": ([ctypes.c_int], ctypes.c_char_p),
@@ -132,6 +138,17 @@ def adafuse_switch_batch_layers(ctx: int, layer_begin: int, n_layers: int, prev:
     _check(lib().adafuse_switch_batch_layers(ctx, int(layer_begin), int(n_layers), prev or None,
                                              cur or None, stream or None),
            "adafuse_switch_batch_layers")
+
+
+def adafuse_set_switch_kernel(ctx: int, kernel: int) -> None:
+    _check(lib().adafuse_set_switch_kernel(ctx, int(kernel)), "adafuse_set_switch_kernel")
+
+
+def adafuse_get_switch_kernel(ctx: int) -> int:
+    k = lib().adafuse_get_switch_kernel(ctx)
+    if k < 0:
+        raise AdafuseError(k, "adafuse_get_switch_kernel")
+    return k
 
 
 def adafuse_get_device_status(ctx: int, stream: int = 0, raise_on_fault: bool = False) -> int:
@@ -210,6 +227,13 @@ class Switcher:
     def switch_layers(self, layer_begin: int, n_layers: int, prev: Optional[int],
                       cur: Optional[int], stream: int = 0) -> None:
         adafuse_switch_batch_layers(self.ctx, layer_begin, n_layers, prev, cur, stream)
+
+    def set_kernel(self, kernel: int) -> None:
+        adafuse_set_switch_kernel(self.ctx, kernel)
+
+    @property
+    def kernel(self) -> int:
+        return adafuse_get_switch_kernel(self.ctx)
 
     def status(self, stream: int = 0) -> int:
         return adafuse_get_device_status(self.ctx, stream)

@@ -14,6 +14,7 @@
 #include "common.cuh"
 #include "pregate.cuh"
 #include "switch_mma.cuh"
+#include "switch_tc.cuh"
 
 using namespace adafuse;
 
@@ -27,6 +28,9 @@ struct adafuse_ctx {
     PairDesc* d_pairs = nullptr;
     TileEntry* d_tiles = nullptr;
     int32_t* d_status = nullptr;
+    CUtensorMap* d_maps = nullptr;  // 3 per pair (W, A, B) when the tensor-core kernel can run
+    int tc_kp = 0;                  // its padded rank (16, 32, 64), 0 = not eligible
+    int kernel = ADAFUSE_KERNEL_AUTO;
 };
 
 namespace {
@@ -97,6 +101,96 @@ int64_t walk_tiles(const adafuse_desc* d, Emit&& emit) {
 }
 
 int kp_class(int r) { return r <= 8 ? 8 : r <= 16 ? 16 : r <= 32 ? 32 : 64; }
+
+// The tensor-core kernel needs TMA-legal strides (rank a multiple of 8).
+int tc_kp_for(int r) { return (r % 8 != 0 || r > 64) ? 0 : r <= 16 ? 16 : r <= 32 ? 32 : 64; }
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+// W [out, in]: box 64 x 128 (cols x rows), 128B swizzle.
+// A [E, r, in]: box 64 x KP x 1, 128B swizzle (rows past r read as zero).
+// B [E, out, r]: box KP x 128 x 1, swizzle = KP*2 bytes (cols past r read as zero).
+bool encode_pair_maps(EncodeTiledFn enc, const PairDesc& pd, int E, int r, int kp,
+                      CUtensorMap out[3]) {
+    const cuuint32_t ones[3] = {1, 1, 1};
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)pd.in, (cuuint64_t)pd.out};
+        const cuuint64_t strides[1] = {(cuuint64_t)pd.in * 2};
+        const cuuint32_t box[2] = {64, 128};
+        if (enc(&out[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (void*)pd.W, dims, strides, box,
+                ones, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return false;
+    }
+    {
+        const cuuint64_t dims[3] = {(cuuint64_t)pd.in, (cuuint64_t)r, (cuuint64_t)E};
+        const cuuint64_t strides[2] = {(cuuint64_t)pd.in * 2, (cuuint64_t)pd.in * r * 2};
+        const cuuint32_t box[3] = {64, (cuuint32_t)kp, 1};
+        if (enc(&out[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, (void*)pd.A, dims, strides, box,
+                ones, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return false;
+    }
+    {
+        const cuuint64_t dims[3] = {(cuuint64_t)r, (cuuint64_t)pd.out, (cuuint64_t)E};
+        const cuuint64_t strides[2] = {(cuuint64_t)r * 2, (cuuint64_t)pd.out * r * 2};
+        const cuuint32_t box[3] = {(cuuint32_t)kp, 128, 1};
+        const CUtensorMapSwizzle sw = kp == 16 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                    : kp == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                               : CU_TENSOR_MAP_SWIZZLE_128B;
+        if (enc(&out[2], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, (void*)pd.B, dims, strides, box,
+                ones, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return false;
+    }
+    return true;
+}
+
+template <int KP>
+cudaError_t launch_tc(const adafuse_ctx* c, int64_t t0, int64_t t1, const adafuse_route* prev,
+                      const adafuse_route* cur, cudaStream_t s) {
+    const int smem = (int)TcConfig<KP>::kSmemBytes;
+    static int configured_for = -1;  // device ordinal the attribute was set on
+    if (configured_for != c->device) {
+        cudaError_t e = cudaFuncSetAttribute(switch_tc_kernel<KP>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        configured_for = c->device;
+    }
+    TcParams prm;
+    prm.pairs = c->d_pairs;
+    prm.tiles = c->d_tiles;
+    prm.maps = c->d_maps;
+    prm.t_begin = t0;
+    prm.t_end = t1;
+    prm.prev = prev;
+    prm.cur = cur;
+    prm.E = c->n_experts;
+    prm.s = c->scale;
+    prm.status = c->d_status;
+    const int64_t n = t1 - t0;
+    const unsigned grid = (unsigned)(n < c->sm_count ? n : c->sm_count);
+    switch_tc_kernel<KP><<<grid, kTcThreads, smem, s>>>(prm);
+    return cudaGetLastError();
+}
 
 }  // namespace
 
@@ -198,6 +292,7 @@ int adafuse_create(adafuse_ctx** out, const adafuse_desc* desc, int device) {
         cudaFree(c->d_pairs);
         cudaFree(c->d_tiles);
         cudaFree(c->d_status);
+        cudaFree(c->d_maps);
         delete c;
         return err == cudaErrorMemoryAllocation ? ADAFUSE_ERR_OUT_OF_MEMORY : cuda_fail(err, what);
     };
@@ -215,6 +310,32 @@ int adafuse_create(adafuse_ctx** out, const adafuse_desc* desc, int device) {
         return fail(e, "cudaMemcpy(tiles)");
     if ((e = cudaMemset(c->d_status, 0, sizeof(int32_t))) != cudaSuccess)
         return fail(e, "cudaMemset(status)");
+
+    // tensor maps for the tensor-core kernel (when the rank allows TMA)
+    c->tc_kp = tc_kp_for(desc->rank);
+    if (c->tc_kp != 0) {
+        EncodeTiledFn enc = encode_tiled_fn();
+        std::vector<CUtensorMap> maps;
+        bool ok = enc != nullptr;
+        if (ok) {
+            try {
+                maps.resize((size_t)npairs * 3);
+            } catch (...) {
+                ok = false;
+            }
+        }
+        for (int64_t i = 0; ok && i < npairs; ++i)
+            ok = encode_pair_maps(enc, pairs[i], desc->n_experts, desc->rank, c->tc_kp, &maps[3 * i]);
+        if (ok) {
+            if ((e = cudaMalloc(&c->d_maps, sizeof(CUtensorMap) * maps.size())) != cudaSuccess)
+                return fail(e, "cudaMalloc(maps)");
+            if ((e = cudaMemcpy(c->d_maps, maps.data(), sizeof(CUtensorMap) * maps.size(),
+                                cudaMemcpyHostToDevice)) != cudaSuccess)
+                return fail(e, "cudaMemcpy(maps)");
+        } else {
+            c->tc_kp = 0;  // fall back to the mma.sync kernel for this context
+        }
+    }
     *out = c;
     return ADAFUSE_OK;
 }
@@ -225,8 +346,26 @@ int adafuse_destroy(adafuse_ctx* ctx) {
     cudaFree(ctx->d_pairs);
     cudaFree(ctx->d_tiles);
     cudaFree(ctx->d_status);
+    cudaFree(ctx->d_maps);
     delete ctx;
     return ADAFUSE_OK;
+}
+
+int adafuse_set_switch_kernel(adafuse_ctx* ctx, int kernel) {
+    if (ctx == nullptr) return ADAFUSE_ERR_INVALID_ARG;
+    if (kernel != ADAFUSE_KERNEL_AUTO && kernel != ADAFUSE_KERNEL_MMA_SYNC &&
+        kernel != ADAFUSE_KERNEL_TCGEN05)
+        return ADAFUSE_ERR_INVALID_ARG;
+    if (kernel == ADAFUSE_KERNEL_TCGEN05 && ctx->tc_kp == 0) return ADAFUSE_ERR_UNSUPPORTED_SHAPE;
+    ctx->kernel = kernel;
+    return ADAFUSE_OK;
+}
+
+int adafuse_get_switch_kernel(adafuse_ctx* ctx) {
+    if (ctx == nullptr) return ADAFUSE_ERR_INVALID_ARG;
+    if (ctx->kernel == ADAFUSE_KERNEL_AUTO)
+        return ctx->tc_kp != 0 ? ADAFUSE_KERNEL_TCGEN05 : ADAFUSE_KERNEL_MMA_SYNC;
+    return ctx->kernel;
 }
 
 int adafuse_pregate(adafuse_ctx* ctx, const float* h, int64_t T, int64_t d, const float* Wr,
@@ -270,6 +409,15 @@ int adafuse_switch_batch_layers(adafuse_ctx* ctx, int32_t layer_begin, int32_t n
     DeviceGuard guard(ctx->device);
     if (!guard.ok) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (adafuse_get_switch_kernel(ctx) == ADAFUSE_KERNEL_TCGEN05) {
+        cudaError_t e = cudaSuccess;
+        switch (ctx->tc_kp) {
+            case 16: e = launch_tc<16>(ctx, t0, t1, prev, cur, s); break;
+            case 32: e = launch_tc<32>(ctx, t0, t1, prev, cur, s); break;
+            default: e = launch_tc<64>(ctx, t0, t1, prev, cur, s); break;
+        }
+        return e == cudaSuccess ? ADAFUSE_OK : cuda_fail(e, "switch launch");
+    }
     const int64_t want = (int64_t)ctx->sm_count * 2;
     const unsigned grid = (unsigned)(t1 - t0 < want ? t1 - t0 : want);
     const int E = ctx->n_experts, r = ctx->rank;

@@ -1,0 +1,326 @@
+// switch_tc.cuh -- fused adapter switch on the 5th-generation tensor cores
+// (tcgen05.mma, accumulators in TMEM), with TMA moving every tile.
+//
+// AdaFuse (gist.science technical summary, section 2-na): one launch walks the
+// segment table and, per 128x128 W tile, applies
+//   W <- bf16_rne(W + sum_e c_e (B_e A_e)),  c_e = s (g_cur(e) - g_prev(e)).
+// The pages' ingredients map onto Blackwell like this:
+//   "segmented"       the tile table; each CTA takes a strided slice of it
+//                     (persistent grid, one CTA per SM);
+//   "gather/concat"   per tile and selected expert, TMA fetches the expert's
+//                     B rows [row0, row0+128) x [0, r) and A columns
+//                     [col0, col0+128) x [0, r) straight from the stacked
+//                     [E, ...] tensors (the expert index is the TMA z
+//                     coordinate); rank r is padded to KP in {16,32,64} by
+//                     TMA's out-of-bounds zero fill;
+//   "parallel GEMM"   one tcgen05.mma chain per expert into its own fp32 TMEM
+//                     accumulator (4 experts x 128 columns = all 512 columns);
+//   "in place"        W tiles go HBM -> smem (TMA, 128B swizzle) -> registers,
+//                     the epilogue adds sum_e c_e acc_e in fp32 and rounds once,
+//                     and TMA stores the tile back over itself;
+//   "prefetch buffer" mbarrier-driven smem rings for W tiles and for operand
+//                     slices, filled ahead of use by a producer warp.
+// Warp roles: warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps
+// 2..9 epilogue (row = 32*(warp%4) + lane, column half = (warp-2)/4).
+// Every wait is bounded: on a timeout the CTA raises ADAFUSE_STATUS_TIMEOUT,
+// stops issuing work, lets in-flight copies drain, frees TMEM and returns.
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+#include "sm100_ptx.cuh"
+
+namespace adafuse {
+
+constexpr int kTcThreads = 320;            // 10 warps
+constexpr int kTcEpiThreads = 256;         // warps 2..9
+constexpr uint32_t kWTileBytes = 128 * 128 * 2;
+constexpr uint32_t kWBoxBytes = kWTileBytes / 2;   // 128 rows x 64 cols
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
+
+template <int KP>
+struct TcConfig {
+    static_assert(KP == 16 || KP == 32 || KP == 64, "KP");
+    static constexpr int kWStages = KP == 64 ? 3 : 4;
+    static constexpr int kOpStages = KP == 16 ? 6 : KP == 32 ? 4 : 3;
+    static constexpr uint32_t kAHalfBytes = KP * 128;      // KP rows x 64 cols bf16
+    static constexpr uint32_t kABytes = 2 * kAHalfBytes;   // KP x 128
+    static constexpr uint32_t kBBytes = 128 * KP * 2;      // 128 x KP
+    static constexpr uint32_t kOpStageBytes = kABytes + kBBytes;
+    static constexpr uint32_t kOpBytes = kOpStages * kOpStageBytes;
+    static constexpr uint32_t kWBytes = kWStages * kWTileBytes;
+    static constexpr uint32_t kBLayout = KP == 16 ? sm100::kSwizzle32B
+                                       : KP == 32 ? sm100::kSwizzle64B
+                                                  : sm100::kSwizzle128B;
+    static constexpr uint32_t kBSbo = 8 * KP * 2;          // 8 rows of the swizzled B slice
+    // barriers + tmem base + abort flag, after the data
+    static constexpr uint32_t kBarBytes = 8 * (3 * kWStages + 2 * kOpStages + 2) + 16;
+    static constexpr uint32_t kSmemBytes = 1024 /*alignment slack*/ + kOpBytes + kWBytes + kBarBytes;
+};
+
+struct TcParams {
+    const PairDesc* pairs;
+    const TileEntry* tiles;
+    const CUtensorMap* maps;  // 3 per pair: W, A, B
+    int64_t t_begin, t_end;
+    const adafuse_route* prev;
+    const adafuse_route* cur;
+    int E;
+    float s;
+    int32_t* status;
+};
+
+__device__ __forceinline__ void decode_tile(const TileEntry* tiles, int64_t i, uint32_t& pair,
+                                            int& row0, int& col0) {
+    const TileEntry te = __ldg(tiles + i);
+    pair = te.x;
+    row0 = (int)(te.y >> 16) * kTile;
+    col0 = (int)(te.y & 0xffffu) * kTile;
+}
+
+template <int KP>
+__global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams p) {
+    using C = TcConfig<KP>;
+    using namespace sm100;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* op_ring = smem;                       // [kOpStages][A (KP x 128) | B (128 x KP)]
+    uint8_t* w_ring = smem + C::kOpBytes;          // [kWStages][box0 | box1]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(w_ring + C::kWBytes);
+    uint64_t* w_full = bars;
+    uint64_t* w_empty = w_full + C::kWStages;
+    uint64_t* op_full = w_empty + C::kWStages;
+    uint64_t* op_empty = op_full + C::kOpStages;
+    uint64_t* acc_full = op_empty + C::kOpStages;
+    uint64_t* acc_empty = acc_full + 1;
+    uint64_t* epi_done = acc_empty + 1;            // [kWStages]: epilogue wrote the tile
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epi_done + C::kWStages);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    Coefs cf;
+    const int st = build_coefs(p.prev, p.cur, p.E, p.s, cf);
+    if (st != 0) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(p.status, st);
+        return;
+    }
+    if (cf.n == 0) return;  // identity switch
+    const int64_t first = p.t_begin + blockIdx.x;
+    if (first >= p.t_end) return;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < C::kWStages; ++i) {
+            mbar_init(&w_full[i], 1);
+            mbar_init(&w_empty[i], 1);
+            mbar_init(&epi_done[i], kTcEpiThreads);
+        }
+        for (int i = 0; i < C::kOpStages; ++i) {
+            mbar_init(&op_full[i], 1);
+            mbar_init(&op_empty[i], 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, kTcEpiThreads / 32);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    auto fail = [&](int where) {
+        if (!*abort_flag) {
+            *abort_flag = 1;
+            atomicOr(p.status, ADAFUSE_STATUS_TIMEOUT);
+        }
+        (void)where;
+    };
+
+    if (warp == 0) {
+        // ---------------- TMA producer ----------------
+        if (lane == 0) {
+            int ws = 0, os = 0;
+            uint32_t wph = 0, oph = 0;
+            uint32_t last_pair = 0xffffffffu;
+            for (int64_t t = first; t < p.t_end && !*abort_flag; t += gridDim.x) {
+                uint32_t pair;
+                int row0, col0;
+                decode_tile(p.tiles, t, pair, row0, col0);
+                const CUtensorMap* mW = p.maps + 3 * (size_t)pair;
+                const CUtensorMap* mA = mW + 1;
+                const CUtensorMap* mB = mW + 2;
+                if (pair != last_pair) {
+                    tensormap_acquire(mW);
+                    tensormap_acquire(mA);
+                    tensormap_acquire(mB);
+                    last_pair = pair;
+                }
+                const bool second = col0 + 64 < __ldg(&p.pairs[pair].in);
+                // W tile
+                if (!mbar_wait_bounded(&w_empty[ws], wph ^ 1, abort_flag, kWaitLimitNs)) { fail(1); break; }
+                uint8_t* wdst = w_ring + (size_t)ws * kWTileBytes;
+                mbar_arrive_expect_tx(&w_full[ws], second ? kWTileBytes : kWBoxBytes);
+                tma_load_2d(wdst, mW, col0, row0, &w_full[ws]);
+                if (second) tma_load_2d(wdst + kWBoxBytes, mW, col0 + 64, row0, &w_full[ws]);
+                if (++ws == C::kWStages) { ws = 0; wph ^= 1; }
+                // operand slices, one stage per selected expert
+                bool ok = true;
+#pragma unroll 1
+                for (int ei = 0; ei < cf.n; ++ei) {
+                    const int e = ei == 0 ? cf.e[0] : ei == 1 ? cf.e[1] : ei == 2 ? cf.e[2] : cf.e[3];
+                    if (!mbar_wait_bounded(&op_empty[os], oph ^ 1, abort_flag, kWaitLimitNs)) { ok = false; break; }
+                    uint8_t* a_dst = op_ring + (size_t)os * C::kOpStageBytes;
+                    uint8_t* b_dst = a_dst + C::kABytes;
+                    mbar_arrive_expect_tx(&op_full[os], C::kBBytes + (second ? 2 : 1) * C::kAHalfBytes);
+                    tma_load_3d(b_dst, mB, 0, row0, e, &op_full[os]);
+                    tma_load_3d(a_dst, mA, col0, 0, e, &op_full[os]);
+                    if (second) tma_load_3d(a_dst + C::kAHalfBytes, mA, col0 + 64, 0, e, &op_full[os]);
+                    if (++os == C::kOpStages) { os = 0; oph ^= 1; }
+                }
+                if (!ok) { fail(2); break; }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            constexpr uint32_t idesc = instr_desc_bf16(128, 128, /*B MN-major*/ 1);
+            int os = 0;
+            uint32_t oph = 0, aph = 0;
+            for (int64_t t = first; t < p.t_end && !*abort_flag; t += gridDim.x) {
+                if (!mbar_wait_bounded(acc_empty, aph ^ 1, abort_flag, kWaitLimitNs)) { fail(3); break; }
+                tc_fence_after();
+                bool ok = true;
+#pragma unroll 1
+                for (int ei = 0; ei < cf.n; ++ei) {
+                    if (!mbar_wait_bounded(&op_full[os], oph, abort_flag, kWaitLimitNs)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a_s = smem_u32(op_ring + (size_t)os * C::kOpStageBytes);
+                    const uint32_t b_s = a_s + C::kABytes;
+#pragma unroll
+                    for (int k = 0; k < KP / 16; ++k) {
+                        // MMA A operand: B_e slice, 128 x KP, K-major, rows swizzled
+                        const uint64_t da = smem_desc(b_s + 32u * k, 16, C::kBSbo, C::kBLayout);
+                        // MMA B operand: A_e slice, KP x 128, N-major, two 64-column halves
+                        const uint64_t db = smem_desc(a_s + 2048u * k, C::kAHalfBytes, 1024, kSwizzle128B);
+                        tc_mma_f16(tmem_base + 128u * ei, da, db, idesc, k > 0 ? 1u : 0u);
+                    }
+                    tc_commit(&op_empty[os]);
+                    if (++os == C::kOpStages) { os = 0; oph ^= 1; }
+                }
+                if (!ok) { fail(4); break; }
+                tc_commit(acc_full);
+                aph ^= 1;
+            }
+        }
+    } else {
+        // ---------------- epilogue ----------------
+        // Every decision that can end the loop is made warp-uniform
+        // (__all_sync / __any_sync) so tcgen05.ld's .sync.aligned form always
+        // sees the whole warp.
+        const int ew = warp - 2;
+        const int quarter = warp & 3;
+        const int half = ew >> 2;
+        const int row = quarter * 32 + lane;
+        const uint32_t t_lane = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(half * 64);
+        const bool storer = (ew == 0 && lane == 0);
+        int ws = 0, prev_ws = -1;
+        uint32_t wph = 0, aph = 0;
+        for (int64_t t = first; t < p.t_end; t += gridDim.x) {
+            if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+            uint32_t pair;
+            int row0, col0;
+            decode_tile(p.tiles, t, pair, row0, col0);
+            // 1) sum_e c_e * acc_e for this thread's row, 64 columns
+            bool ok = mbar_wait_bounded(acc_full, aph, abort_flag, kWaitLimitNs);
+            if (!__all_sync(0xffffffffu, ok)) { fail(5); break; }
+            aph ^= 1;
+            tc_fence_after();
+            float tot[64];
+#pragma unroll
+            for (int i = 0; i < 64; ++i) tot[i] = 0.f;
+#pragma unroll
+            for (int ei = 0; ei < 4; ++ei) {
+                if (ei < cf.n) {
+                    const float c = cf.c[ei];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        float v[16];
+                        tmem_ld16(t_lane + 128u * ei + 16u * j, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) tot[16 * j + i] = __fmaf_rn(c, v[i], tot[16 * j + i]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty);
+
+            // 2) W tile: smem (128B-swizzled rows of 64 columns) -> +dW -> smem
+            ok = mbar_wait_bounded(&w_full[ws], wph, abort_flag, kWaitLimitNs);
+            if (!__all_sync(0xffffffffu, ok)) { fail(6); break; }
+            uint8_t* box = w_ring + (size_t)ws * kWTileBytes + (size_t)half * kWBoxBytes;
+            uint8_t* rowp = box + row * 128;
+#pragma unroll
+            for (int c8 = 0; c8 < 8; ++c8) {
+                uint4* q = reinterpret_cast<uint4*>(rowp + ((c8 ^ (row & 7)) << 4));
+                uint4 w = *q;
+                uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float lo = __uint_as_float(wv[j] << 16) + tot[8 * c8 + 2 * j];
+                    const float hi = __uint_as_float(wv[j] & 0xffff0000u) + tot[8 * c8 + 2 * j + 1];
+                    const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+                    wv[j] = *reinterpret_cast<const uint32_t*>(&b);
+                }
+                *q = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+            }
+            fence_async_smem();
+            mbar_arrive(&epi_done[ws]);
+            // 3) one thread stores the tile back over itself once all 256 wrote
+            if (storer) {
+                if (!mbar_wait_bounded(&epi_done[ws], wph, abort_flag, kWaitLimitNs)) {
+                    fail(7);
+                } else {
+                    const CUtensorMap* mW = p.maps + 3 * (size_t)pair;
+                    const bool second = col0 + 64 < __ldg(&p.pairs[pair].in);
+                    uint8_t* wsrc = w_ring + (size_t)ws * kWTileBytes;
+                    tma_store_2d(mW, wsrc, col0, row0);
+                    if (second) tma_store_2d(mW, wsrc + kWBoxBytes, col0 + 64, row0);
+                    bulk_commit();
+                    bulk_wait_read<1>();           // the previous tile's store has read smem
+                    if (prev_ws >= 0) mbar_arrive(&w_empty[prev_ws]);
+                    prev_ws = ws;
+                }
+            }
+            if (++ws == C::kWStages) { ws = 0; wph ^= 1; }
+        }
+        if (storer) {
+            bulk_wait<0>();
+            if (prev_ws >= 0) mbar_arrive(&w_empty[prev_ws]);
+        }
+    }
+
+    // teardown: after an abort give in-flight TMA copies and MMAs time to land
+    __syncwarp();
+    __syncthreads();
+    if (*abort_flag) {
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 200000ull) { }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, 512);
+    }
+}
+
+}  // namespace adafuse
