@@ -208,6 +208,21 @@ def run_reference(args):
 # --------------------------------------------------------------------------
 # our arm
 
+def reduce_over_ranks(total_ms, n_units, world, device="cpu"):
+    """Whole-job timing: the slowest rank's device time and the units (real
+    switches) all ranks processed.  Every rank takes the same collective
+    steps; world == 1 takes none."""
+    import torch
+    import torch.distributed as dist
+    if world <= 1:
+        return float(total_ms), float(n_units)
+    mx = torch.tensor([float(total_ms)], dtype=torch.float64, device=device)
+    sm = torch.tensor([float(n_units)], dtype=torch.float64, device=device)
+    dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+    dist.all_reduce(sm, op=dist.ReduceOp.SUM)
+    return float(mx[0]), float(sm[0])
+
+
 def run_ours(args):
     import numpy as np
     import torch
@@ -302,16 +317,7 @@ def run_ours(args):
             n_real += 1
         p = t
 
-    # max over ranks
-    tm = torch.tensor([total_ms, float(n_real)], dtype=torch.float64, device="cuda")
-    if world > 1:
-        mx = tm.clone()
-        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
-        tot_real = tm[1:].clone()
-        dist.all_reduce(tot_real, op=dist.ReduceOp.SUM)
-        max_ms, all_real = float(mx[0]), float(tot_real[0])
-    else:
-        max_ms, all_real = total_ms, float(n_real)
+    max_ms, all_real = reduce_over_ranks(total_ms, n_real, world, device="cuda")
     value = all_real * w_bytes / (max_ms / 1000.0) / 1e9
 
     # e2e through the public API with host buffers
@@ -337,10 +343,8 @@ def run_ours(args):
         torch.cuda.synchronize()
         barrier()
         e_ms = ev0.elapsed_time(ev1)
-        et = torch.tensor([e_ms], dtype=torch.float64, device="cuda")
-        if world > 1:
-            dist.all_reduce(et, op=dist.ReduceOp.MAX)
-        e2e = {"value": round(world * args.steps * w_bytes / (float(et[0]) / 1000) / 1e9, 2),
+        e_max, e_units = reduce_over_ranks(e_ms, args.steps, world, device="cuda")
+        e2e = {"value": round(e_units * w_bytes / (e_max / 1000) / 1e9, 2),
                "unit": "GB/s", "h2d_bytes_per_step": cfg.d * 4, "d2h_bytes_per_step": 16}
 
     peak, peak_kind = measured_peaks()

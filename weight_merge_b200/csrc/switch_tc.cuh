@@ -20,8 +20,9 @@
 //                     and TMA stores the tile back over itself;
 //   "prefetch buffer" mbarrier-driven smem rings for W tiles and for operand
 //                     slices, filled ahead of use by a producer warp.
-// Warp roles: warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps
-// 2..9 epilogue (row = 32*(warp%4) + lane, column half = (warp-2)/4).
+// Warp roles: warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warp 2
+// TMA store of finished tiles, warps 3..18 epilogue (row = 32*(warp%4) +
+// lane, 32-column group = (warp-3)/4).
 // Every wait is bounded: on a timeout the CTA raises ADAFUSE_STATUS_TIMEOUT,
 // stops issuing work, lets in-flight copies drain, frees TMEM and returns.
 #pragma once
@@ -33,8 +34,9 @@
 
 namespace adafuse {
 
-constexpr int kTcThreads = 320;            // 10 warps
-constexpr int kTcEpiThreads = 256;         // warps 2..9
+constexpr int kTcThreads = 608;            // 19 warps
+constexpr int kTcEpiWarp0 = 3;             // first epilogue warp
+constexpr int kTcEpiThreads = 512;         // warps 3..18
 constexpr uint32_t kWTileBytes = 128 * 128 * 2;
 constexpr uint32_t kWBoxBytes = kWTileBytes / 2;   // 128 rows x 64 cols
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
@@ -42,7 +44,7 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
 template <int KP>
 struct TcConfig {
     static_assert(KP == 16 || KP == 32 || KP == 64, "KP");
-    static constexpr int kWStages = KP == 64 ? 3 : 4;
+    static constexpr int kWStages = KP == 64 ? 3 : KP == 32 ? 4 : 5;
     static constexpr int kOpStages = KP == 16 ? 6 : KP == 32 ? 4 : 3;
     static constexpr uint32_t kAHalfBytes = KP * 128;      // KP rows x 64 cols bf16
     static constexpr uint32_t kABytes = 2 * kAHalfBytes;   // KP x 128
@@ -224,87 +226,90 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
         // Every decision that can end the loop is made warp-uniform
         // (__all_sync / __any_sync) so tcgen05.ld's .sync.aligned form always
         // sees the whole warp.
-        const int ew = warp - 2;
-        const int quarter = warp & 3;
-        const int half = ew >> 2;
-        const int row = quarter * 32 + lane;
-        const uint32_t t_lane = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(half * 64);
-        const bool storer = (ew == 0 && lane == 0);
-        int ws = 0, prev_ws = -1;
-        uint32_t wph = 0, aph = 0;
-        for (int64_t t = first; t < p.t_end; t += gridDim.x) {
-            if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
-            uint32_t pair;
-            int row0, col0;
-            decode_tile(p.tiles, t, pair, row0, col0);
-            // 1) sum_e c_e * acc_e for this thread's row, 64 columns
-            bool ok = mbar_wait_bounded(acc_full, aph, abort_flag, kWaitLimitNs);
-            if (!__all_sync(0xffffffffu, ok)) { fail(5); break; }
-            aph ^= 1;
-            tc_fence_after();
-            float tot[64];
-#pragma unroll
-            for (int i = 0; i < 64; ++i) tot[i] = 0.f;
-#pragma unroll
-            for (int ei = 0; ei < 4; ++ei) {
-                if (ei < cf.n) {
-                    const float c = cf.c[ei];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        float v[16];
-                        tmem_ld16(t_lane + 128u * ei + 16u * j, v);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) tot[16 * j + i] = __fmaf_rn(c, v[i], tot[16 * j + i]);
-                    }
-                }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(acc_empty);
-
-            // 2) W tile: smem (128B-swizzled rows of 64 columns) -> +dW -> smem
-            ok = mbar_wait_bounded(&w_full[ws], wph, abort_flag, kWaitLimitNs);
-            if (!__all_sync(0xffffffffu, ok)) { fail(6); break; }
-            uint8_t* box = w_ring + (size_t)ws * kWTileBytes + (size_t)half * kWBoxBytes;
-            uint8_t* rowp = box + row * 128;
-#pragma unroll
-            for (int c8 = 0; c8 < 8; ++c8) {
-                uint4* q = reinterpret_cast<uint4*>(rowp + ((c8 ^ (row & 7)) << 4));
-                uint4 w = *q;
-                uint32_t wv[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float lo = __uint_as_float(wv[j] << 16) + tot[8 * c8 + 2 * j];
-                    const float hi = __uint_as_float(wv[j] & 0xffff0000u) + tot[8 * c8 + 2 * j + 1];
-                    const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
-                    wv[j] = *reinterpret_cast<const uint32_t*>(&b);
-                }
-                *q = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-            }
-            fence_async_smem();
-            mbar_arrive(&epi_done[ws]);
-            // 3) one thread stores the tile back over itself once all 256 wrote
-            if (storer) {
-                if (!mbar_wait_bounded(&epi_done[ws], wph, abort_flag, kWaitLimitNs)) {
-                    fail(7);
-                } else {
+        if (warp == 2) {
+            // ---- store warp: TMA-stores each finished tile over itself and
+            // frees its smem stage as soon as the store has read it.
+            if (lane == 0) {
+                int ws = 0;
+                uint32_t wph = 0;
+                for (int64_t t = first; t < p.t_end && !*abort_flag; t += gridDim.x) {
+                    uint32_t pair;
+                    int row0, col0;
+                    decode_tile(p.tiles, t, pair, row0, col0);
+                    if (!mbar_wait_bounded(&epi_done[ws], wph, abort_flag, kWaitLimitNs)) { fail(7); break; }
                     const CUtensorMap* mW = p.maps + 3 * (size_t)pair;
                     const bool second = col0 + 64 < __ldg(&p.pairs[pair].in);
                     uint8_t* wsrc = w_ring + (size_t)ws * kWTileBytes;
                     tma_store_2d(mW, wsrc, col0, row0);
                     if (second) tma_store_2d(mW, wsrc + kWBoxBytes, col0 + 64, row0);
                     bulk_commit();
-                    bulk_wait_read<1>();           // the previous tile's store has read smem
-                    if (prev_ws >= 0) mbar_arrive(&w_empty[prev_ws]);
-                    prev_ws = ws;
+                    bulk_wait_read<0>();
+                    mbar_arrive(&w_empty[ws]);
+                    if (++ws == C::kWStages) { ws = 0; wph ^= 1; }
                 }
+                bulk_wait<0>();
             }
-            if (++ws == C::kWStages) { ws = 0; wph ^= 1; }
-        }
-        if (storer) {
-            bulk_wait<0>();
-            if (prev_ws >= 0) mbar_arrive(&w_empty[prev_ws]);
+        } else {
+            const int ew = warp - kTcEpiWarp0;      // 0..15
+            const int quarter = warp & 3;           // TMEM lanes this warp may read
+            const int cgrp = ew >> 2;               // 32-column group 0..3
+            const int half = cgrp >> 1;             // which 64-column TMA box
+            const int row = quarter * 32 + lane;
+            const uint32_t t_lane = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(cgrp * 32);
+            int ws = 0;
+            uint32_t wph = 0, aph = 0;
+            for (int64_t t = first; t < p.t_end; t += gridDim.x) {
+                if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+                // 1) sum_e c_e * acc_e for this thread's row, 32 columns
+                bool ok = mbar_wait_bounded(acc_full, aph, abort_flag, kWaitLimitNs);
+                if (!__all_sync(0xffffffffu, ok)) { fail(5); break; }
+                aph ^= 1;
+                tc_fence_after();
+                float tot[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) tot[i] = 0.f;
+#pragma unroll
+                for (int ei = 0; ei < 4; ++ei) {
+                    if (ei < cf.n) {
+                        const float c = cf.c[ei];
+                        float v[32];
+                        tmem_ld32(t_lane + 128u * ei, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) tot[i] = __fmaf_rn(c, v[i], tot[i]);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(acc_empty);
+
+                // 2) W: smem (128B-swizzled rows of 64 columns) -> +dW -> smem
+                ok = mbar_wait_bounded(&w_full[ws], wph, abort_flag, kWaitLimitNs);
+                if (!__all_sync(0xffffffffu, ok)) { fail(6); break; }
+                uint8_t* rowp = w_ring + (size_t)ws * kWTileBytes + (size_t)half * kWBoxBytes + row * 128;
+                uint4 w[4];
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    const int chunk = (cgrp & 1) * 4 + c4;   // 16-byte chunk within the 128-byte row
+                    w[c4] = lds128(rowp + ((chunk ^ (row & 7)) << 4));
+                }
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    uint32_t wv[4] = {w[c4].x, w[c4].y, w[c4].z, w[c4].w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float lo = __uint_as_float(wv[j] << 16) + tot[8 * c4 + 2 * j];
+                        const float hi = __uint_as_float(wv[j] & 0xffff0000u) + tot[8 * c4 + 2 * j + 1];
+                        const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+                        wv[j] = *reinterpret_cast<const uint32_t*>(&b);
+                    }
+                    const int chunk = (cgrp & 1) * 4 + c4;
+                    sts128(rowp + ((chunk ^ (row & 7)) << 4), make_uint4(wv[0], wv[1], wv[2], wv[3]));
+                }
+                fence_async_smem();
+                mbar_arrive(&epi_done[ws]);
+                if (++ws == C::kWStages) { ws = 0; wph ^= 1; }
+            }
         }
     }
 
