@@ -193,6 +193,45 @@ ADAFUSE_API int adafuse_get_device_status(adafuse_ctx* ctx, void* stream, int32_
 ADAFUSE_API int adafuse_segment_table(const adafuse_desc* desc, int32_t* entries,
                           int64_t capacity, int64_t* count);
 
+/* ---- allocation-free switch -------------------------------------------- */
+#define ADAFUSE_NOALLOC_SCRATCH_BYTES 65536  /* static device scratch per GPU */
+#define ADAFUSE_NOALLOC_MAX_WEIGHTS   1638   /* (layer, target) weights it can hold */
+
+/* The fused switch for callers that cannot allocate device memory.  The
+ * AdaFuse pages have no counterpart to this entry point: it exists for
+ * deployment, not for the method.
+ *
+ * adafuse_create calls cudaMalloc for its tile table, weight descriptors and
+ * status word.  Some callers cannot: a serving engine that has handed all
+ * free HBM to its own memory pool (a later cudaMalloc fails or fragments the
+ * pool), or a decode loop that must not stall on cudaMalloc's implicit
+ * device synchronisation.  This call needs no context and allocates nothing
+ * -- no cudaMalloc, no cudaFree, no allocating library routine.  It performs
+ * the same switch as adafuse_switch over every (layer, target) of `desc`, on
+ * the current device, with the mma.sync kernel, and gives the same result to
+ * within the documented rounding.
+ *
+ * Scratch: one file-scope static device array of
+ * ADAFUSE_NOALLOC_SCRATCH_BYTES (64 KiB), which every GPU that loads this
+ * library holds until the process exits.  Each call rewrites it with the
+ * weight table of `desc`, so ALL calls share it: two calls whose work
+ * overlaps on the GPU (different streams, or threads without ordering)
+ * race and may switch the wrong weights.  Calls on one stream are ordered
+ * and safe.  The first call on each device also looks up the array's device
+ * address (once per device); make that first call before any stream capture.
+ *
+ * Arguments: desc as for adafuse_create (host memory, read during the call
+ * only; its device pointers must stay valid until the switch completes);
+ * prev / cur as for adafuse_switch; status: optional 4-byte-aligned device
+ * int32 that the call first sets to 0 and the kernel then ORs
+ * ADAFUSE_STATUS_* bits into (a bad route writes no W); stream: cudaStream_t.
+ * Returns ADAFUSE_ERR_UNSUPPORTED_SHAPE when desc has more than
+ * ADAFUSE_NOALLOC_MAX_WEIGHTS weights (or a shape adafuse_create rejects),
+ * INVALID_ARG / UNSUPPORTED_DEVICE / CUDA otherwise as adafuse_create and
+ * adafuse_switch do.  Asynchronous like adafuse_switch. */
+ADAFUSE_API int adafuse_switch_noalloc(const adafuse_desc* desc, const adafuse_route* prev,
+                                       const adafuse_route* cur, int32_t* status, void* stream);
+
 /* Tile edge of the segment table (128). */
 ADAFUSE_API int adafuse_tile_size(void);
 
