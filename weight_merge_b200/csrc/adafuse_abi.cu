@@ -67,7 +67,7 @@ int check_desc(const adafuse_desc* d, bool need_pointers) {
     if (d->rank < 1 || d->rank > 64) return ADAFUSE_ERR_UNSUPPORTED_SHAPE;
     if (!std::isfinite(d->alpha)) return ADAFUSE_ERR_INVALID_ARG;
     const int64_t n = (int64_t)d->n_layers * d->n_targets;
-    if (n > (int64_t)1 << 30) return ADAFUSE_ERR_UNSUPPORTED_SHAPE;
+    if (n > (int64_t)1 << 30) return ADAFUSE_ERR_UNSUPPORTED_SHAPE;  // pair index < 2^31
     for (int64_t i = 0; i < n; ++i) {
         const adafuse_target& t = d->targets[i];
         if (t.out <= 0 || t.in <= 0) return ADAFUSE_ERR_INVALID_ARG;
@@ -186,6 +186,7 @@ cudaError_t launch_tc(const adafuse_ctx* c, int64_t t0, int64_t t1, const adafus
     prm.E = c->n_experts;
     prm.s = c->scale;
     prm.status = c->d_status;
+    prm.b_bulk = c->rank == 8 ? 1 : 0;
     const int64_t n = t1 - t0;
     const unsigned grid = (unsigned)(n < c->sm_count ? n : c->sm_count);
     switch_tc_kernel<KP><<<grid, kTcThreads, smem, s>>>(prm);
@@ -276,8 +277,10 @@ int adafuse_create(adafuse_ctx** out, const adafuse_desc* desc, int device) {
     try {
         tiles.reserve((size_t)walk_tiles(desc, [](int, int, int64_t, int64_t, int64_t) {}));
         walk_tiles(desc, [&](int l, int k, int64_t i, int64_t j, int64_t) {
+            const adafuse_target& tg = desc->targets[(int64_t)l * desc->n_targets + k];
             TileEntry te;
             te.x = (uint32_t)((int64_t)l * desc->n_targets + k);
+            if (j * kTile + 64 < tg.in) te.x |= kTileWideBit;
             te.y = (uint32_t)((i << 16) | j);
             tiles.push_back(te);
             c->layer_tile_begin[(size_t)l + 1] = (int64_t)tiles.size();

@@ -24,9 +24,12 @@ struct PairDesc {
 };
 
 // One segment-table entry: which weight, which 128x128 tile of it.
-//   x = index into the PairDesc array
+//   x = index into the PairDesc array | (1 << 31) when the tile's second
+//       64-column half starts inside the weight (col0 + 64 < in)
 //   y = (row tile << 16) | col tile
 using TileEntry = uint2;
+constexpr uint32_t kTileWideBit = 0x80000000u;
+constexpr uint32_t kTilePairMask = 0x7fffffffu;
 
 // The union of the previous and the current route, as coefficients:
 // c_e = s * (g_cur(e) - g_prev(e)) for each distinct expert, zeros dropped.

@@ -94,7 +94,7 @@ struct TileCoord {
 __device__ __forceinline__ TileCoord load_tile(const PairDesc* __restrict__ pairs,
                                                const TileEntry* __restrict__ tiles, int64_t i) {
     const TileEntry te = __ldg(tiles + i);
-    const PairDesc* pd = pairs + te.x;
+    const PairDesc* pd = pairs + (te.x & kTilePairMask);
     TileCoord tc;
     tc.W = pd->W;
     tc.A = pd->A;

@@ -20,9 +20,11 @@
 //                     and TMA stores the tile back over itself;
 //   "prefetch buffer" mbarrier-driven smem rings for W tiles and for operand
 //                     slices, filled ahead of use by a producer warp.
-// Warp roles: warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warp 2
-// TMA store of finished tiles, warps 3..18 epilogue (row = 32*(warp%4) +
-// lane, 32-column group = (warp-3)/4).
+// Warp roles: warp 0 W-tile producer (TMA), warp 1 TMEM owner
+// + MMA issuer, warp 2 TMA store of finished tiles, warp 3 operand-slice
+// producer, warps 4..19 epilogue (row = 32*(warp%4) + lane, 32-column group =
+// (warp-4)/4).  The two producers are separate so that W loads run ahead of
+// the MMA-paced operand ring.
 // Every wait is bounded: on a timeout the CTA raises ADAFUSE_STATUS_TIMEOUT,
 // stops issuing work, lets in-flight copies drain, frees TMEM and returns.
 #pragma once
@@ -34,9 +36,9 @@
 
 namespace adafuse {
 
-constexpr int kTcThreads = 608;            // 19 warps
-constexpr int kTcEpiWarp0 = 3;             // first epilogue warp
-constexpr int kTcEpiThreads = 512;         // warps 3..18
+constexpr int kTcThreads = 640;            // 20 warps
+constexpr int kTcEpiWarp0 = 4;             // first epilogue warp
+constexpr int kTcEpiThreads = 512;         // warps 4..19
 constexpr uint32_t kWTileBytes = 128 * 128 * 2;
 constexpr uint32_t kWBoxBytes = kWTileBytes / 2;   // 128 rows x 64 cols
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
@@ -71,14 +73,32 @@ struct TcParams {
     int E;
     float s;
     int32_t* status;
+    // rank == 8: an expert's 128 B rows are one contiguous 2 KB block that is
+    // already the no-swizzle K-major core-matrix layout, so it is fetched with
+    // one bulk copy (16 full 128-byte lines) instead of a 128-row tensor box
+    // of 16-byte rows.
+    int b_bulk;
 };
 
-__device__ __forceinline__ void decode_tile(const TileEntry* tiles, int64_t i, uint32_t& pair,
-                                            int& row0, int& col0) {
-    const TileEntry te = __ldg(tiles + i);
-    pair = te.x;
-    row0 = (int)(te.y >> 16) * kTile;
-    col0 = (int)(te.y & 0xffffu) * kTile;
+// Tile entries are fetched one iteration ahead (the loops below keep the next
+// entry in a register), so no tile waits on a dependent global load.
+__device__ __forceinline__ TileEntry fetch_tile(const TileEntry* tiles, int64_t i, int64_t end) {
+    return i < end ? __ldg(tiles + i) : make_uint2(0u, 0u);
+}
+
+struct TileInfo {
+    uint32_t pair;
+    int row0, col0;
+    bool wide;  // second 64-column half starts inside the weight
+};
+
+__device__ __forceinline__ TileInfo decode_tile(TileEntry te) {
+    TileInfo ti;
+    ti.pair = te.x & kTilePairMask;
+    ti.wide = (te.x & kTileWideBit) != 0;
+    ti.row0 = (int)(te.y >> 16) * kTile;
+    ti.col0 = (int)(te.y & 0xffffu) * kTile;
+    return ti;
 }
 
 template <int KP>
@@ -146,33 +166,61 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
     };
 
     if (warp == 0) {
-        // ---------------- TMA producer ----------------
+        // ---------------- W producer: tiles into the W ring ----
+        // Runs ahead of everything else, limited only by free W stages.
         if (lane == 0) {
-            int ws = 0, os = 0;
-            uint32_t wph = 0, oph = 0;
+            int ws = 0;
+            uint32_t wph = 0;
             uint32_t last_pair = 0xffffffffu;
+            TileEntry te_next = fetch_tile(p.tiles, first, p.t_end);
             for (int64_t t = first; t < p.t_end && !*abort_flag; t += gridDim.x) {
-                uint32_t pair;
-                int row0, col0;
-                decode_tile(p.tiles, t, pair, row0, col0);
-                const CUtensorMap* mW = p.maps + 3 * (size_t)pair;
-                const CUtensorMap* mA = mW + 1;
-                const CUtensorMap* mB = mW + 2;
-                if (pair != last_pair) {
+                const TileInfo ti = decode_tile(te_next);
+                te_next = fetch_tile(p.tiles, t + gridDim.x, p.t_end);
+                const CUtensorMap* mW = p.maps + 3 * (size_t)ti.pair;
+                if (ti.pair != last_pair) {
                     tensormap_acquire(mW);
+                    last_pair = ti.pair;
+                }
+                if (!mbar_wait_bounded(&w_empty[ws], wph ^ 1, abort_flag, kWaitLimitNs)) { fail(1); break; }
+                uint8_t* wdst = w_ring + (size_t)ws * kWTileBytes;
+                mbar_arrive_expect_tx(&w_full[ws], ti.wide ? kWTileBytes : kWBoxBytes);
+                tma_load_2d(wdst, mW, ti.col0, ti.row0, &w_full[ws]);
+                if (ti.wide) tma_load_2d(wdst + kWBoxBytes, mW, ti.col0 + 64, ti.row0, &w_full[ws]);
+                if (++ws == C::kWStages) { ws = 0; wph ^= 1; }
+                if (t + gridDim.x < p.t_end && (te_next.x & kTilePairMask) != ti.pair)
+                    tensormap_prefetch(p.maps + 3 * (size_t)(te_next.x & kTilePairMask));
+            }
+        }
+    } else if (warp == 3) {
+        // ---------------- operand producer: per tile and expert, the B-row and
+        // A-column slices into the operand ring (paced by the MMA warp) ----
+        if (lane == 0) {
+            int os = 0;
+            uint32_t oph = 0;
+            uint32_t last_pair = 0xffffffffu;
+            TileEntry te_next = fetch_tile(p.tiles, first, p.t_end);
+            for (int64_t t = first; t < p.t_end && !*abort_flag; t += gridDim.x) {
+                const TileInfo ti = decode_tile(te_next);
+                te_next = fetch_tile(p.tiles, t + gridDim.x, p.t_end);
+                const uint32_t pair = ti.pair;
+                const int row0 = ti.row0, col0 = ti.col0;
+                const CUtensorMap* mA = p.maps + 3 * (size_t)pair + 1;
+                const CUtensorMap* mB = mA + 1;
+                if (pair != last_pair) {
                     tensormap_acquire(mA);
                     tensormap_acquire(mB);
                     last_pair = pair;
                 }
-                const bool second = col0 + 64 < __ldg(&p.pairs[pair].in);
-                // W tile
-                if (!mbar_wait_bounded(&w_empty[ws], wph ^ 1, abort_flag, kWaitLimitNs)) { fail(1); break; }
-                uint8_t* wdst = w_ring + (size_t)ws * kWTileBytes;
-                mbar_arrive_expect_tx(&w_full[ws], second ? kWTileBytes : kWBoxBytes);
-                tma_load_2d(wdst, mW, col0, row0, &w_full[ws]);
-                if (second) tma_load_2d(wdst + kWBoxBytes, mW, col0 + 64, row0, &w_full[ws]);
-                if (++ws == C::kWStages) { ws = 0; wph ^= 1; }
-                // operand slices, one stage per selected expert
+                const bool second = ti.wide;
+                int out_rows = 128;
+                const uint16_t* Bbase = nullptr;
+                int out = 0;
+                if (p.b_bulk) {
+                    const PairDesc& pd = p.pairs[pair];
+                    out = pd.out;
+                    Bbase = pd.B;
+                    out_rows = out - row0 < 128 ? out - row0 : 128;
+                }
                 bool ok = true;
 #pragma unroll 1
                 for (int ei = 0; ei < cf.n; ++ei) {
@@ -180,13 +228,26 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
                     if (!mbar_wait_bounded(&op_empty[os], oph ^ 1, abort_flag, kWaitLimitNs)) { ok = false; break; }
                     uint8_t* a_dst = op_ring + (size_t)os * C::kOpStageBytes;
                     uint8_t* b_dst = a_dst + C::kABytes;
-                    mbar_arrive_expect_tx(&op_full[os], C::kBBytes + (second ? 2 : 1) * C::kAHalfBytes);
-                    tma_load_3d(b_dst, mB, 0, row0, e, &op_full[os]);
+                    if (p.b_bulk) {
+                        // rows past the weight's end are not fetched (their
+                        // products only reach accumulator rows never stored)
+                        const uint32_t bbytes = (uint32_t)out_rows * 16u;
+                        mbar_arrive_expect_tx(&op_full[os], bbytes + (second ? 2 : 1) * C::kAHalfBytes);
+                        bulk_load(b_dst, Bbase + ((size_t)e * out + row0) * 8, bbytes, &op_full[os]);
+                    } else {
+                        mbar_arrive_expect_tx(&op_full[os], C::kBBytes + (second ? 2 : 1) * C::kAHalfBytes);
+                        tma_load_3d(b_dst, mB, 0, row0, e, &op_full[os]);
+                    }
                     tma_load_3d(a_dst, mA, col0, 0, e, &op_full[os]);
                     if (second) tma_load_3d(a_dst + C::kAHalfBytes, mA, col0 + 64, 0, e, &op_full[os]);
                     if (++os == C::kOpStages) { os = 0; oph ^= 1; }
                 }
                 if (!ok) { fail(2); break; }
+                if (t + gridDim.x < p.t_end && (te_next.x & kTilePairMask) != pair) {
+                    const CUtensorMap* nm = p.maps + 3 * (size_t)(te_next.x & kTilePairMask);
+                    tensormap_prefetch(nm + 1);
+                    tensormap_prefetch(nm + 2);
+                }
             }
         }
     } else if (warp == 1) {
@@ -208,7 +269,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
 #pragma unroll
                     for (int k = 0; k < KP / 16; ++k) {
                         // MMA A operand: B_e slice, 128 x KP, K-major, rows swizzled
-                        const uint64_t da = smem_desc(b_s + 32u * k, 16, C::kBSbo, C::kBLayout);
+                        // rank 8 (bulk-copied, plain core-matrix layout): the
+                        // second 8-deep K chunk re-reads the first (LBO 0); the
+                        // matching A rows 8..15 are TMA zero fill, so it adds 0
+                        const uint64_t da = p.b_bulk
+                            ? smem_desc(b_s, 0, 128, kSwizzleNone)
+                            : smem_desc(b_s + 32u * k, 16, C::kBSbo, C::kBLayout);
                         // MMA B operand: A_e slice, KP x 128, N-major, two 64-column halves
                         const uint64_t db = smem_desc(a_s + 2048u * k, C::kAHalfBytes, 1024, kSwizzle128B);
                         tc_mma_f16(tmem_base + 128u * ei, da, db, idesc, k > 0 ? 1u : 0u);
@@ -232,13 +298,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
             if (lane == 0) {
                 int ws = 0;
                 uint32_t wph = 0;
+                TileEntry te_next = fetch_tile(p.tiles, first, p.t_end);
                 for (int64_t t = first; t < p.t_end && !*abort_flag; t += gridDim.x) {
-                    uint32_t pair;
-                    int row0, col0;
-                    decode_tile(p.tiles, t, pair, row0, col0);
+                    const TileInfo ti = decode_tile(te_next);
+                    te_next = fetch_tile(p.tiles, t + gridDim.x, p.t_end);
+                    const int row0 = ti.row0, col0 = ti.col0;
                     if (!mbar_wait_bounded(&epi_done[ws], wph, abort_flag, kWaitLimitNs)) { fail(7); break; }
-                    const CUtensorMap* mW = p.maps + 3 * (size_t)pair;
-                    const bool second = col0 + 64 < __ldg(&p.pairs[pair].in);
+                    const CUtensorMap* mW = p.maps + 3 * (size_t)ti.pair;
+                    const bool second = ti.wide;
                     uint8_t* wsrc = w_ring + (size_t)ws * kWTileBytes;
                     tma_store_2d(mW, wsrc, col0, row0);
                     if (second) tma_store_2d(mW, wsrc + kWBoxBytes, col0 + 64, row0);
