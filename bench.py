@@ -50,9 +50,43 @@ def parse():
                     help="switch kernel: tensor-core (tc), mma.sync (mma), or auto")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--traffic-gb", type=float, default=None,
-                    help="ncu dram bytes (read+write) of one switch launch, GB")
     return ap.parse_args()
+
+
+def kernel_source_hash():
+    """sha256 over the CUDA sources and the ABI header (identifies the kernels
+    an ncu capture was taken on)."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "weight_merge_b200", "csrc")
+    files = sorted(os.path.join(csrc, f) for f in os.listdir(csrc) if f.endswith((".cu", ".cuh")))
+    for f in files + [os.path.join(ROOT, "include", "adafuse.h")]:
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode())
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(kernel_name, workload):
+    """DRAM bytes (read + write) per full launch from a committed ncu summary
+    in profiles/, or None when none matches the current kernel sources."""
+    d = os.path.join(ROOT, "profiles")
+    if not os.path.isdir(d):
+        return None
+    want = kernel_source_hash()
+    for f in sorted(os.listdir(d)):
+        if not f.endswith(".md"):
+            continue
+        meta = {}
+        for line in open(os.path.join(d, f)):
+            if line.startswith("- ") and ": " in line:
+                k, v = line[2:].strip().split(": ", 1)
+                meta[k.strip("`")] = v.strip().strip("`")
+        if (meta.get("kernel") == kernel_name and meta.get("workload") == workload
+                and meta.get("kernel-source-sha256") == want
+                and "dram-bytes-per-full-launch" in meta):
+            return int(meta["dram-bytes-per-full-launch"])
+    return None
 
 
 def measured_peaks():
@@ -382,7 +416,7 @@ def run_ours(args):
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                          "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "peak_kind": peak_kind,
-                         "traffic": (round(args.traffic_gb * 1e9) if args.traffic_gb else None),
+                         "traffic": profiled_traffic(kernel_name, cfg.name),
                          "kernel": kernel_name},
             "cpu_baseline": cpu,
             "e2e": e2e,
