@@ -48,6 +48,8 @@ def parse():
                     help="override the layer count (small cases for ncu captures)")
     ap.add_argument("--kernel", choices=["auto", "mma", "tc"], default="auto",
                     help="switch kernel: tensor-core (tc), mma.sync (mma), or auto")
+    ap.add_argument("--mode", choices=["switch", "rebase"], default="switch",
+                    help="in-place switch (prev -> cur) or re-base from a pristine copy W0")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -287,6 +289,9 @@ def run_ours(args):
                    "tc": B.ADAFUSE_KERNEL_TCGEN05}[args.kernel])
     kernel_name = {B.ADAFUSE_KERNEL_MMA_SYNC: "switch_mma_kernel",
                    B.ADAFUSE_KERNEL_TCGEN05: "switch_tc_kernel"}[sw.kernel]
+    rebase = args.mode == "rebase"
+    if rebase:
+        sw.set_base([w.clone() for w in model.W])
     T = cfg.n_tokens
     h = wl.make_hidden(cfg, T=T, device="cuda")
     routes = torch.zeros((T, 4), dtype=torch.int32, device="cuda")
@@ -298,10 +303,16 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
 
+    def do_switch(prev_t, t):
+        if rebase:
+            sw.rebase(B.Switcher.route_ptr(routes, t), sh)
+        else:
+            sw.switch(B.Switcher.route_ptr(routes, prev_t), B.Switcher.route_ptr(routes, t), sh)
+
     def step(k, prev_t):
         t = k % T
         sw.pregate(h[t:t + 1], model.Wr, routes[t:t + 1], sh)
-        sw.switch(B.Switcher.route_ptr(routes, prev_t), B.Switcher.route_ptr(routes, t), sh)
+        do_switch(prev_t, t)
         return t
 
     # warm-up
@@ -328,7 +339,7 @@ def run_ours(args):
             st_start[k].record(stream)
             sw.pregate(h[t:t + 1], model.Wr, routes[t:t + 1], sh)
             sw_start[k].record(stream)
-            sw.switch(B.Switcher.route_ptr(routes, prev_t), B.Switcher.route_ptr(routes, t), sh)
+            do_switch(prev_t, t)
             sw_end[k].record(stream)
             prev_t = t
         t_end.record(stream)
@@ -347,7 +358,7 @@ def run_ours(args):
     p = (args.warmup - 1) % T if args.warmup > 0 else None
     for k in range(args.steps):
         t = (args.warmup + k) % T
-        if p is None or not np.array_equal(r_np[p], r_np[t]):
+        if rebase or p is None or not np.array_equal(r_np[p], r_np[t]):
             n_real += 1
         p = t
 
@@ -370,7 +381,7 @@ def run_ours(args):
             t = (args.warmup + args.steps + k) % T
             h_dev.copy_(h_host[t:t + 1], non_blocking=True)
             sw.pregate(h_dev, model.Wr, routes[t:t + 1], sh)
-            sw.switch(B.Switcher.route_ptr(routes, pe), B.Switcher.route_ptr(routes, t), sh)
+            do_switch(pe, t)
             r_host.copy_(routes[t:t + 1], non_blocking=True)
             pe = t
         ev1.record(stream)
@@ -407,6 +418,7 @@ def run_ours(args):
                 "w_bytes_per_switch": w_bytes,
                 "l2": "inputs larger than L2 (W read+write per switch >> 126 MB), no flush",
                 "parallelism": f"replicas x{world}",
+                "mode": args.mode,
             },
             "switch_ms_p50": round(sw_sorted[len(sw_sorted) // 2], 4),
             "switch_ms_p90": round(sw_sorted[min(len(sw_sorted) - 1, int(0.9 * len(sw_sorted)))], 4),

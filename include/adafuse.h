@@ -181,6 +181,32 @@ ADAFUSE_API int adafuse_set_switch_kernel(adafuse_ctx* ctx, int kernel);
  * ADAFUSE_KERNEL_TCGEN05), or a negative code. */
 ADAFUSE_API int adafuse_get_switch_kernel(adafuse_ctx* ctx);
 
+/* ---- re-base switch ------------------------------------------------------
+ * A variant of the switch that the AdaFuse pages do not describe (they merge
+ * in place, section 2-na): the caller keeps a pristine copy W0 of every
+ * targeted weight, and each call writes W <- bf16_rne(W0 + s*sum_{e in cur}
+ * g_e B_e A_e).  It moves the same bytes as the in-place switch (W0 read, W
+ * written), needs no previous route, cannot drift, and costs a second copy
+ * of the targeted weights in device memory. */
+
+/* Register the pristine weights: W0 is a host array of n_layers*n_targets
+ * device pointers, one per (layer, target) in the same order as the
+ * context's targets, each [out, in] bf16, 16-byte aligned, distinct from W.
+ * The caller owns W0 and must not modify it while re-base calls may run.
+ * Builds device-side descriptors (allocates; not for the hot path) and
+ * synchronises the device.  Calling it again replaces the base. */
+ADAFUSE_API int adafuse_set_base(adafuse_ctx* ctx, const void* const* W0);
+
+/* W <- bf16_rne(W0 + s*sum_{e in cur} g_e B_e A_e) for every layer and
+ * target, one kernel launch on `stream`.  cur: 16-byte aligned device route
+ * or NULL (then W <- W0).  INVALID_ARG without a registered base.  Bad
+ * routes behave as in adafuse_switch (status bit, nothing written). */
+ADAFUSE_API int adafuse_rebase(adafuse_ctx* ctx, const adafuse_route* cur, void* stream);
+
+/* As adafuse_rebase, restricted to layers [layer_begin, layer_begin + n_layers). */
+ADAFUSE_API int adafuse_rebase_layers(adafuse_ctx* ctx, int32_t layer_begin, int32_t n_layers,
+                                      const adafuse_route* cur, void* stream);
+
 /* Synchronise `stream`, read the device status word into *status, then
  * clear it.  Returns ADAFUSE_ERR_DEVICE_FAULT when the word was non-zero,
  * ADAFUSE_OK otherwise. */

@@ -13,6 +13,7 @@ from .binding import (  # noqa: F401
     ADAFUSE_KERNEL_AUTO, ADAFUSE_KERNEL_MMA_SYNC, ADAFUSE_KERNEL_TCGEN05, AdafuseError, Route, Target, Desc,
     lib, library_path, adafuse_create, adafuse_destroy, adafuse_pregate, adafuse_switch,
     adafuse_switch_batch_layers, adafuse_get_device_status, adafuse_set_switch_kernel,
-    adafuse_get_switch_kernel, adafuse_segment_table,
+    adafuse_get_switch_kernel, adafuse_segment_table, adafuse_set_base, adafuse_rebase,
+    adafuse_rebase_layers,
     adafuse_tile_size, adafuse_strerror, adafuse_last_error, Switcher,
 )

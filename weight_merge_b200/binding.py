@@ -80,6 +80,9 @@ def lib() -> ctypes.CDLL:
         "adafuse_switch_batch_layers": ([P, i32, i32, P, P, P], ctypes.c_int),
         "adafuse_get_device_status": ([P, P, ctypes.POINTER(i32)], ctypes.c_int),
         "adafuse_set_switch_kernel": ([P, ctypes.c_int], ctypes.c_int),
+        "adafuse_set_base": ([P, ctypes.POINTER(P)], ctypes.c_int),
+        "adafuse_rebase": ([P, P, P], ctypes.c_int),
+        "adafuse_rebase_layers": ([P, i32, i32, P, P], ctypes.c_int),
         "adafuse_get_switch_kernel": ([P], ctypes.c_int),
         "adafuse_segment_table": ([ctypes.POINTER(Desc), P, i64, ctypes.POINTER(i64)], ctypes.c_int),
         "adafuse_tile_size": ([], ctypes.c_int),
@@ -138,6 +141,21 @@ def adafuse_switch_batch_layers(ctx: int, layer_begin: int, n_layers: int, prev:
     _check(lib().adafuse_switch_batch_layers(ctx, int(layer_begin), int(n_layers), prev or None,
                                              cur or None, stream or None),
            "adafuse_switch_batch_layers")
+
+
+def adafuse_set_base(ctx: int, W0: Sequence[int]) -> None:
+    arr = (ctypes.c_void_p * len(W0))(*W0)
+    _check(lib().adafuse_set_base(ctx, arr), "adafuse_set_base")
+
+
+def adafuse_rebase(ctx: int, cur: Optional[int], stream: int = 0) -> None:
+    _check(lib().adafuse_rebase(ctx, cur or None, stream or None), "adafuse_rebase")
+
+
+def adafuse_rebase_layers(ctx: int, layer_begin: int, n_layers: int, cur: Optional[int],
+                          stream: int = 0) -> None:
+    _check(lib().adafuse_rebase_layers(ctx, int(layer_begin), int(n_layers), cur or None,
+                                       stream or None), "adafuse_rebase_layers")
 
 
 def adafuse_set_switch_kernel(ctx: int, kernel: int) -> None:
@@ -227,6 +245,18 @@ class Switcher:
     def switch_layers(self, layer_begin: int, n_layers: int, prev: Optional[int],
                       cur: Optional[int], stream: int = 0) -> None:
         adafuse_switch_batch_layers(self.ctx, layer_begin, n_layers, prev, cur, stream)
+
+    def set_base(self, W0) -> None:
+        """W0: list of tensors (pristine copies of W, same order); kept alive here."""
+        self._base = list(W0)
+        adafuse_set_base(self.ctx, [w.data_ptr() for w in self._base])
+
+    def rebase(self, cur: Optional[int], stream: int = 0) -> None:
+        adafuse_rebase(self.ctx, cur, stream)
+
+    def rebase_layers(self, layer_begin: int, n_layers: int, cur: Optional[int],
+                      stream: int = 0) -> None:
+        adafuse_rebase_layers(self.ctx, layer_begin, n_layers, cur, stream)
 
     def set_kernel(self, kernel: int) -> None:
         adafuse_set_switch_kernel(self.ctx, kernel)

@@ -31,6 +31,9 @@ struct adafuse_ctx {
     CUtensorMap* d_maps = nullptr;  // 3 per pair (W, A, B) when the tensor-core kernel can run
     int tc_kp = 0;                  // its padded rank (16, 32, 64), 0 = not eligible
     int kernel = ADAFUSE_KERNEL_AUTO;
+    std::vector<PairDesc> h_pairs;  // host copy of d_pairs (re-base pointers are patched in)
+    CUtensorMap* d_w0_maps = nullptr;  // 1 per pair on the re-base source W0
+    bool has_base = false;
 };
 
 namespace {
@@ -166,7 +169,7 @@ bool encode_pair_maps(EncodeTiledFn enc, const PairDesc& pd, int E, int r, int k
 
 template <int KP>
 cudaError_t launch_tc(const adafuse_ctx* c, int64_t t0, int64_t t1, const adafuse_route* prev,
-                      const adafuse_route* cur, cudaStream_t s) {
+                      const adafuse_route* cur, cudaStream_t s, bool rebase) {
     const int smem = (int)TcConfig<KP>::kSmemBytes;
     static int configured_for = -1;  // device ordinal the attribute was set on
     if (configured_for != c->device) {
@@ -187,6 +190,8 @@ cudaError_t launch_tc(const adafuse_ctx* c, int64_t t0, int64_t t1, const adafus
     prm.s = c->scale;
     prm.status = c->d_status;
     prm.b_bulk = c->rank == 8 ? 1 : 0;
+    prm.rebase = rebase ? 1 : 0;
+    prm.w0_maps = c->d_w0_maps;
     const int64_t n = t1 - t0;
     const unsigned grid = (unsigned)(n < c->sm_count ? n : c->sm_count);
     switch_tc_kernel<KP><<<grid, kTcThreads, smem, s>>>(prm);
@@ -265,6 +270,7 @@ int adafuse_create(adafuse_ctx** out, const adafuse_desc* desc, int device) {
     for (int64_t i = 0; i < npairs; ++i) {
         const adafuse_target& t = desc->targets[i];
         pairs[i].W = static_cast<uint16_t*>(t.W);
+        pairs[i].W0 = nullptr;
         pairs[i].A = static_cast<const uint16_t*>(t.A);
         pairs[i].B = static_cast<const uint16_t*>(t.B);
         pairs[i].out = (int32_t)t.out;
@@ -290,6 +296,12 @@ int adafuse_create(adafuse_ctx** out, const adafuse_desc* desc, int device) {
         return ADAFUSE_ERR_OUT_OF_MEMORY;
     }
     c->n_tiles = (int64_t)tiles.size();
+    try {
+        c->h_pairs = pairs;
+    } catch (...) {
+        delete c;
+        return ADAFUSE_ERR_OUT_OF_MEMORY;
+    }
 
     auto fail = [&](cudaError_t err, const char* what) {
         cudaFree(c->d_pairs);
@@ -350,6 +362,7 @@ int adafuse_destroy(adafuse_ctx* ctx) {
     cudaFree(ctx->d_tiles);
     cudaFree(ctx->d_status);
     cudaFree(ctx->d_maps);
+    cudaFree(ctx->d_w0_maps);
     delete ctx;
     return ADAFUSE_OK;
 }
@@ -399,9 +412,14 @@ int adafuse_pregate(adafuse_ctx* ctx, const float* h, int64_t T, int64_t d, cons
     return e == cudaSuccess ? ADAFUSE_OK : cuda_fail(e, "pregate launch");
 }
 
-int adafuse_switch_batch_layers(adafuse_ctx* ctx, int32_t layer_begin, int32_t n_layers,
-                                const adafuse_route* prev, const adafuse_route* cur,
-                                void* stream) {
+}  // extern "C"
+
+namespace {
+
+// One switch launch over layers [layer_begin, layer_begin + n_layers): in
+// place (prev, cur) or, with rebase, W <- rne(W0 + dW_cur).
+int launch_switch(adafuse_ctx* ctx, int32_t layer_begin, int32_t n_layers,
+                  const adafuse_route* prev, const adafuse_route* cur, void* stream, bool rebase) {
     if (ctx == nullptr || n_layers < 0 || layer_begin < 0) return ADAFUSE_ERR_INVALID_ARG;
     if ((int64_t)layer_begin + n_layers > ctx->n_layers) return ADAFUSE_ERR_INVALID_ARG;
     if (!aligned16(prev) || !aligned16(cur)) return ADAFUSE_ERR_INVALID_ARG;
@@ -415,9 +433,9 @@ int adafuse_switch_batch_layers(adafuse_ctx* ctx, int32_t layer_begin, int32_t n
     if (adafuse_get_switch_kernel(ctx) == ADAFUSE_KERNEL_TCGEN05) {
         cudaError_t e = cudaSuccess;
         switch (ctx->tc_kp) {
-            case 16: e = launch_tc<16>(ctx, t0, t1, prev, cur, s); break;
-            case 32: e = launch_tc<32>(ctx, t0, t1, prev, cur, s); break;
-            default: e = launch_tc<64>(ctx, t0, t1, prev, cur, s); break;
+            case 16: e = launch_tc<16>(ctx, t0, t1, prev, cur, s, rebase); break;
+            case 32: e = launch_tc<32>(ctx, t0, t1, prev, cur, s, rebase); break;
+            default: e = launch_tc<64>(ctx, t0, t1, prev, cur, s, rebase); break;
         }
         return e == cudaSuccess ? ADAFUSE_OK : cuda_fail(e, "switch launch");
     }
@@ -425,26 +443,97 @@ int adafuse_switch_batch_layers(adafuse_ctx* ctx, int32_t layer_begin, int32_t n
     const unsigned grid = (unsigned)(t1 - t0 < want ? t1 - t0 : want);
     const int E = ctx->n_experts, r = ctx->rank;
     const float sc = ctx->scale;
+    const int rb = rebase ? 1 : 0;
     switch (kp_class(r)) {
         case 8:
             switch_mma_kernel<8><<<grid, kSwitchThreads, 0, s>>>(ctx->d_pairs, ctx->d_tiles, t0, t1,
-                                                                 prev, cur, E, r, sc, ctx->d_status);
+                                                                 prev, cur, E, r, sc, ctx->d_status, rb);
             break;
         case 16:
             switch_mma_kernel<16><<<grid, kSwitchThreads, 0, s>>>(ctx->d_pairs, ctx->d_tiles, t0, t1,
-                                                                  prev, cur, E, r, sc, ctx->d_status);
+                                                                  prev, cur, E, r, sc, ctx->d_status, rb);
             break;
         case 32:
             switch_mma_kernel<32><<<grid, kSwitchThreads, 0, s>>>(ctx->d_pairs, ctx->d_tiles, t0, t1,
-                                                                  prev, cur, E, r, sc, ctx->d_status);
+                                                                  prev, cur, E, r, sc, ctx->d_status, rb);
             break;
         default:
             switch_mma_kernel<64><<<grid, kSwitchThreads, 0, s>>>(ctx->d_pairs, ctx->d_tiles, t0, t1,
-                                                                  prev, cur, E, r, sc, ctx->d_status);
+                                                                  prev, cur, E, r, sc, ctx->d_status, rb);
             break;
     }
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? ADAFUSE_OK : cuda_fail(e, "switch launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+int adafuse_switch_batch_layers(adafuse_ctx* ctx, int32_t layer_begin, int32_t n_layers,
+                                const adafuse_route* prev, const adafuse_route* cur,
+                                void* stream) {
+    return launch_switch(ctx, layer_begin, n_layers, prev, cur, stream, false);
+}
+
+int adafuse_set_base(adafuse_ctx* ctx, const void* const* W0) {
+    if (ctx == nullptr || W0 == nullptr) return ADAFUSE_ERR_INVALID_ARG;
+    const size_t n = ctx->h_pairs.size();
+    for (size_t i = 0; i < n; ++i)
+        if (W0[i] == nullptr || !aligned16(W0[i]) || W0[i] == ctx->h_pairs[i].W)
+            return ADAFUSE_ERR_INVALID_ARG;
+    DeviceGuard guard(ctx->device);
+    if (!guard.ok) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
+    std::vector<PairDesc> pairs;
+    std::vector<CUtensorMap> maps;
+    try {
+        pairs = ctx->h_pairs;
+        if (ctx->tc_kp != 0) maps.resize(n);
+    } catch (...) {
+        return ADAFUSE_ERR_OUT_OF_MEMORY;
+    }
+    for (size_t i = 0; i < n; ++i) pairs[i].W0 = static_cast<const uint16_t*>(W0[i]);
+    if (ctx->tc_kp != 0) {
+        EncodeTiledFn enc = encode_tiled_fn();
+        if (enc == nullptr) return ADAFUSE_ERR_CUDA;
+        for (size_t i = 0; i < n; ++i) {
+            PairDesc src = pairs[i];
+            src.W = const_cast<uint16_t*>(src.W0);
+            CUtensorMap three[3];
+            if (!encode_pair_maps(enc, src, ctx->n_experts, ctx->rank, ctx->tc_kp, three))
+                return ADAFUSE_ERR_CUDA;
+            maps[i] = three[0];
+        }
+    }
+    // everything the kernels may still be reading is replaced only after the
+    // device is idle with respect to this context's stream-ordered work
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+    if (ctx->tc_kp != 0 && ctx->d_w0_maps == nullptr) {
+        e = cudaMalloc(&ctx->d_w0_maps, sizeof(CUtensorMap) * n);
+        if (e != cudaSuccess)
+            return e == cudaErrorMemoryAllocation ? ADAFUSE_ERR_OUT_OF_MEMORY : cuda_fail(e, "cudaMalloc(w0 maps)");
+    }
+    if (ctx->tc_kp != 0) {
+        e = cudaMemcpy(ctx->d_w0_maps, maps.data(), sizeof(CUtensorMap) * n, cudaMemcpyHostToDevice);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(w0 maps)");
+    }
+    e = cudaMemcpy(ctx->d_pairs, pairs.data(), sizeof(PairDesc) * n, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(pairs)");
+    ctx->h_pairs.swap(pairs);
+    ctx->has_base = true;
+    return ADAFUSE_OK;
+}
+
+int adafuse_rebase_layers(adafuse_ctx* ctx, int32_t layer_begin, int32_t n_layers,
+                          const adafuse_route* cur, void* stream) {
+    if (ctx == nullptr || !ctx->has_base) return ADAFUSE_ERR_INVALID_ARG;
+    return launch_switch(ctx, layer_begin, n_layers, nullptr, cur, stream, true);
+}
+
+int adafuse_rebase(adafuse_ctx* ctx, const adafuse_route* cur, void* stream) {
+    if (ctx == nullptr) return ADAFUSE_ERR_INVALID_ARG;
+    return adafuse_rebase_layers(ctx, 0, ctx->n_layers, cur, stream);
 }
 
 int adafuse_switch(adafuse_ctx* ctx, const adafuse_route* prev, const adafuse_route* cur,

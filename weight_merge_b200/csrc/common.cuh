@@ -14,9 +14,10 @@ constexpr int kTile = 128;
 
 // One (layer, target) weight as the kernels see it.
 struct PairDesc {
-    uint16_t* W;        // [out, in] bf16 bits
-    const uint16_t* A;  // [E, r, in]
-    const uint16_t* B;  // [E, out, r]
+    uint16_t* W;         // [out, in] bf16 bits
+    const uint16_t* A;   // [E, r, in]
+    const uint16_t* B;   // [E, out, r]
+    const uint16_t* W0;  // [out, in] pristine base for the re-base switch (or null)
     int32_t out;
     int32_t in;
     int32_t layer;

@@ -66,6 +66,7 @@ __device__ __forceinline__ TileCoord tile_of(const Entry* tab, int w, int64_t t)
     const int64_t ct = (en.in + kTile - 1) / kTile;
     TileCoord tc;
     tc.W = en.W;
+    tc.Wsrc = en.W;
     tc.A = en.A;
     tc.B = en.B;
     tc.out = en.out;

@@ -86,17 +86,20 @@ __device__ __forceinline__ uint32_t f2_to_bf2(float lo, float hi) {
 struct TileCoord {
     const uint16_t* A;
     const uint16_t* B;
-    uint16_t* W;
+    uint16_t* W;          // written
+    const uint16_t* Wsrc; // read: W itself, or the pristine base when re-basing
     int out, in;
     int row0, col0;
 };
 
 __device__ __forceinline__ TileCoord load_tile(const PairDesc* __restrict__ pairs,
-                                               const TileEntry* __restrict__ tiles, int64_t i) {
+                                               const TileEntry* __restrict__ tiles, int64_t i,
+                                               bool rebase) {
     const TileEntry te = __ldg(tiles + i);
     const PairDesc* pd = pairs + (te.x & kTilePairMask);
     TileCoord tc;
     tc.W = pd->W;
+    tc.Wsrc = rebase ? pd->W0 : pd->W;
     tc.A = pd->A;
     tc.B = pd->B;
     tc.out = pd->out;
@@ -107,18 +110,20 @@ __device__ __forceinline__ TileCoord load_tile(const PairDesc* __restrict__ pair
 }
 
 // KP: per-expert contraction depth rounded up to 8, 16, 32 or 64.
+// rebase: read W from the pristine base W0 instead of W itself (prev is null),
+// so W <- rne(W0 + dW_cur); then even an empty route writes (it copies W0).
 template <int KP>
 __global__ void __launch_bounds__(kSwitchThreads, 2)
 switch_mma_kernel(const PairDesc* __restrict__ pairs, const TileEntry* __restrict__ tiles,
                   int64_t t_begin, int64_t t_end, const adafuse_route* prev,
-                  const adafuse_route* cur, int E, int r, float s, int32_t* status) {
+                  const adafuse_route* cur, int E, int r, float s, int32_t* status, int rebase) {
     Coefs cf;
     const int st = build_coefs(prev, cur, E, s, cf);
     if (st != 0) {
         if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(status, st);
         return;
     }
-    if (cf.n == 0) return;  // identity switch: nothing to write
+    if (cf.n == 0 && !rebase) return;  // identity switch: nothing to write
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
@@ -127,7 +132,7 @@ switch_mma_kernel(const PairDesc* __restrict__ pairs, const TileEntry* __restric
 
     int64_t tile = t_begin + blockIdx.x;
     if (tile >= t_end) return;
-    TileCoord tc = load_tile(pairs, tiles, tile);
+    TileCoord tc = load_tile(pairs, tiles, tile, rebase != 0);
 
     uint4 wv[4][2];
 #pragma unroll
@@ -137,7 +142,7 @@ switch_mma_kernel(const PairDesc* __restrict__ pairs, const TileEntry* __restric
             const int row = tc.row0 + 16 * warp + g + 8 * hh;
             const int col = tc.col0 + 32 * cg + 8 * t;
             wv[cg][hh] = (row < tc.out && col < tc.in)
-                             ? ld_stream_16(tc.W + (int64_t)row * tc.in + col)
+                             ? ld_stream_16(tc.Wsrc + (int64_t)row * tc.in + col)
                              : make_uint4(0u, 0u, 0u, 0u);
         }
 
@@ -145,7 +150,7 @@ switch_mma_kernel(const PairDesc* __restrict__ pairs, const TileEntry* __restric
         const int64_t next = tile + gridDim.x;
         const bool has_next = next < t_end;
         TileCoord tn = tc;
-        if (has_next) tn = load_tile(pairs, tiles, next);
+        if (has_next) tn = load_tile(pairs, tiles, next, rebase != 0);
 
         const int rowA = tc.row0 + 16 * warp + g;  // rows rowA and rowA + 8
         const bool okA0 = rowA < tc.out, okA1 = rowA + 8 < tc.out;
@@ -229,7 +234,7 @@ switch_mma_kernel(const PairDesc* __restrict__ pairs, const TileEntry* __restric
                     const int nrow = tn.row0 + 16 * warp + g + 8 * hh;
                     const int ncol = tn.col0 + 32 * cg + 8 * t;
                     wv[cg][hh] = (nrow < tn.out && ncol < tn.in)
-                                     ? ld_stream_16(tn.W + (int64_t)nrow * tn.in + ncol)
+                                     ? ld_stream_16(tn.Wsrc + (int64_t)nrow * tn.in + ncol)
                                      : make_uint4(0u, 0u, 0u, 0u);
                 }
             }

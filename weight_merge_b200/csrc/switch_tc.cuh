@@ -78,6 +78,11 @@ struct TcParams {
     // one bulk copy (16 full 128-byte lines) instead of a 128-row tensor box
     // of 16-byte rows.
     int b_bulk;
+    // re-base switch: W tiles are read through w0_maps (one map per pair, on
+    // the pristine base W0) and written through the W maps, prev is null, and
+    // a tile is written even when no expert is selected (it copies W0).
+    int rebase;
+    const CUtensorMap* w0_maps;
 };
 
 // Tile entries are fetched one iteration ahead (the loops below keep the next
@@ -127,7 +132,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
         if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(p.status, st);
         return;
     }
-    if (cf.n == 0) return;  // identity switch
+    if (cf.n == 0 && !p.rebase) return;  // identity switch
     const int64_t first = p.t_begin + blockIdx.x;
     if (first >= p.t_end) return;
 
@@ -176,7 +181,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
             for (int64_t t = first; t < p.t_end && !*abort_flag; t += gridDim.x) {
                 const TileInfo ti = decode_tile(te_next);
                 te_next = fetch_tile(p.tiles, t + gridDim.x, p.t_end);
-                const CUtensorMap* mW = p.maps + 3 * (size_t)ti.pair;
+                const CUtensorMap* mW = p.rebase ? p.w0_maps + ti.pair : p.maps + 3 * (size_t)ti.pair;
                 if (ti.pair != last_pair) {
                     tensormap_acquire(mW);
                     last_pair = ti.pair;
@@ -187,8 +192,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
                 tma_load_2d(wdst, mW, ti.col0, ti.row0, &w_full[ws]);
                 if (ti.wide) tma_load_2d(wdst + kWBoxBytes, mW, ti.col0 + 64, ti.row0, &w_full[ws]);
                 if (++ws == C::kWStages) { ws = 0; wph ^= 1; }
-                if (t + gridDim.x < p.t_end && (te_next.x & kTilePairMask) != ti.pair)
-                    tensormap_prefetch(p.maps + 3 * (size_t)(te_next.x & kTilePairMask));
+                if (t + gridDim.x < p.t_end && (te_next.x & kTilePairMask) != ti.pair) {
+                    const uint32_t np = te_next.x & kTilePairMask;
+                    tensormap_prefetch(p.rebase ? p.w0_maps + np : p.maps + 3 * (size_t)np);
+                }
             }
         }
     } else if (warp == 3) {
