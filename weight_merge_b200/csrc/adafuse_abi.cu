@@ -146,7 +146,9 @@ bool encode_pair_maps(EncodeTiledFn enc, const PairDesc& pd, int E, int r, int k
     {
         const cuuint64_t dims[3] = {(cuuint64_t)pd.in, (cuuint64_t)r, (cuuint64_t)E};
         const cuuint64_t strides[2] = {(cuuint64_t)pd.in * 2, (cuuint64_t)pd.in * r * 2};
-        const cuuint32_t box[3] = {64, (cuuint32_t)kp, 1};
+        // rank 8 fetches exactly its 8 rows; other ranks a KP-row box whose
+        // rows past r read as zero
+        const cuuint32_t box[3] = {64, (cuuint32_t)(r == 8 ? 8 : kp), 1};
         if (enc(&out[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, (void*)pd.A, dims, strides, box,
                 ones, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                 CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
@@ -167,13 +169,13 @@ bool encode_pair_maps(EncodeTiledFn enc, const PairDesc& pd, int E, int r, int k
     return true;
 }
 
-template <int KP>
+template <int KP, bool BBULK>
 cudaError_t launch_tc(const adafuse_ctx* c, int64_t t0, int64_t t1, const adafuse_route* prev,
                       const adafuse_route* cur, cudaStream_t s, bool rebase) {
-    const int smem = (int)TcConfig<KP>::kSmemBytes;
+    const int smem = (int)TcConfig<KP, BBULK>::kSmemBytes;
     static int configured_for = -1;  // device ordinal the attribute was set on
     if (configured_for != c->device) {
-        cudaError_t e = cudaFuncSetAttribute(switch_tc_kernel<KP>,
+        cudaError_t e = cudaFuncSetAttribute(switch_tc_kernel<KP, BBULK>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         configured_for = c->device;
@@ -189,12 +191,11 @@ cudaError_t launch_tc(const adafuse_ctx* c, int64_t t0, int64_t t1, const adafus
     prm.E = c->n_experts;
     prm.s = c->scale;
     prm.status = c->d_status;
-    prm.b_bulk = c->rank == 8 ? 1 : 0;
     prm.rebase = rebase ? 1 : 0;
     prm.w0_maps = c->d_w0_maps;
     const int64_t n = t1 - t0;
     const unsigned grid = (unsigned)(n < c->sm_count ? n : c->sm_count);
-    switch_tc_kernel<KP><<<grid, kTcThreads, smem, s>>>(prm);
+    switch_tc_kernel<KP, BBULK><<<grid, kTcThreads, smem, s>>>(prm);
     return cudaGetLastError();
 }
 
@@ -432,11 +433,14 @@ int launch_switch(adafuse_ctx* ctx, int32_t layer_begin, int32_t n_layers,
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (adafuse_get_switch_kernel(ctx) == ADAFUSE_KERNEL_TCGEN05) {
         cudaError_t e = cudaSuccess;
-        switch (ctx->tc_kp) {
-            case 16: e = launch_tc<16>(ctx, t0, t1, prev, cur, s, rebase); break;
-            case 32: e = launch_tc<32>(ctx, t0, t1, prev, cur, s, rebase); break;
-            default: e = launch_tc<64>(ctx, t0, t1, prev, cur, s, rebase); break;
-        }
+        if (ctx->rank == 8)
+            e = launch_tc<16, true>(ctx, t0, t1, prev, cur, s, rebase);
+        else if (ctx->tc_kp == 16)
+            e = launch_tc<16, false>(ctx, t0, t1, prev, cur, s, rebase);
+        else if (ctx->tc_kp == 32)
+            e = launch_tc<32, false>(ctx, t0, t1, prev, cur, s, rebase);
+        else
+            e = launch_tc<64, false>(ctx, t0, t1, prev, cur, s, rebase);
         return e == cudaSuccess ? ADAFUSE_OK : cuda_fail(e, "switch launch");
     }
     const int64_t want = (int64_t)ctx->sm_count * 2;

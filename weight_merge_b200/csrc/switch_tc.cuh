@@ -43,16 +43,25 @@ constexpr uint32_t kWTileBytes = 128 * 128 * 2;
 constexpr uint32_t kWBoxBytes = kWTileBytes / 2;   // 128 rows x 64 cols
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
 
-template <int KP>
+// KP: per-expert contraction depth (rank padded to 16, 32 or 64).
+// BBULK: rank 8.  Its B rows (128 x 8) are one contiguous 2 KB block already in
+// the plain core-matrix layout, fetched with one bulk copy; its A columns are
+// an 8-row TMA box per 64-column half, and the MMA's second 8-deep K group
+// reads a shared zero block instead (through the descriptor's K-group stride),
+// so each operand stage is 4 KB and the W ring gets a sixth stage.
+template <int KP, bool BBULK>
 struct TcConfig {
     static_assert(KP == 16 || KP == 32 || KP == 64, "KP");
-    static constexpr int kWStages = KP == 64 ? 3 : KP == 32 ? 4 : 5;
+    static_assert(!BBULK || KP == 16, "the bulk path is rank 8");
+    static constexpr int kWStages = BBULK ? 6 : KP == 64 ? 3 : KP == 32 ? 4 : 5;
     static constexpr int kOpStages = KP == 16 ? 6 : KP == 32 ? 4 : 3;
-    static constexpr uint32_t kAHalfBytes = KP * 128;      // KP rows x 64 cols bf16
-    static constexpr uint32_t kABytes = 2 * kAHalfBytes;   // KP x 128
-    static constexpr uint32_t kBBytes = 128 * KP * 2;      // 128 x KP
+    static constexpr uint32_t kARows = BBULK ? 8 : KP;             // A rows fetched
+    static constexpr uint32_t kAHalfBytes = kARows * 128;          // rows x 64 cols bf16
+    static constexpr uint32_t kABytes = 2 * kAHalfBytes;
+    static constexpr uint32_t kBBytes = BBULK ? 128 * 8 * 2 : 128 * KP * 2;  // 128 x r|KP
     static constexpr uint32_t kOpStageBytes = kABytes + kBBytes;
     static constexpr uint32_t kOpBytes = kOpStages * kOpStageBytes;
+    static constexpr uint32_t kZeroBytes = BBULK ? 2048 : 0;      // K rows 8..15 of both halves
     static constexpr uint32_t kWBytes = kWStages * kWTileBytes;
     static constexpr uint32_t kBLayout = KP == 16 ? sm100::kSwizzle32B
                                        : KP == 32 ? sm100::kSwizzle64B
@@ -60,7 +69,10 @@ struct TcConfig {
     static constexpr uint32_t kBSbo = 8 * KP * 2;          // 8 rows of the swizzled B slice
     // barriers + tmem base + abort flag, after the data
     static constexpr uint32_t kBarBytes = 8 * (3 * kWStages + 2 * kOpStages + 2) + 16;
-    static constexpr uint32_t kSmemBytes = 1024 /*alignment slack*/ + kOpBytes + kWBytes + kBarBytes;
+    static constexpr uint32_t kSmemBytes =
+        1024 /*alignment slack*/ + kOpBytes + kZeroBytes + kWBytes + kBarBytes;
+    static_assert(kSmemBytes <= 232448, "shared memory");
+    static_assert(kOpStageBytes % 1024 == 0 && kAHalfBytes % 1024 == 0, "swizzle atoms stay aligned");
 };
 
 struct TcParams {
@@ -73,11 +85,6 @@ struct TcParams {
     int E;
     float s;
     int32_t* status;
-    // rank == 8: an expert's 128 B rows are one contiguous 2 KB block that is
-    // already the no-swizzle K-major core-matrix layout, so it is fetched with
-    // one bulk copy (16 full 128-byte lines) instead of a 128-row tensor box
-    // of 16-byte rows.
-    int b_bulk;
     // re-base switch: W tiles are read through w0_maps (one map per pair, on
     // the pristine base W0) and written through the W maps, prev is null, and
     // a tile is written even when no expert is selected (it copies W0).
@@ -106,15 +113,16 @@ __device__ __forceinline__ TileInfo decode_tile(TileEntry te) {
     return ti;
 }
 
-template <int KP>
+template <int KP, bool BBULK>
 __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams p) {
-    using C = TcConfig<KP>;
+    using C = TcConfig<KP, BBULK>;
     using namespace sm100;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* op_ring = smem;                       // [kOpStages][A (KP x 128) | B (128 x KP)]
-    uint8_t* w_ring = smem + C::kOpBytes;          // [kWStages][box0 | box1]
+    uint8_t* op_ring = smem;                       // [kOpStages][A (rows x 128) | B (128 x r|KP)]
+    uint8_t* zero_blk = smem + C::kOpBytes;        // rank 8: zero K rows 8..15
+    uint8_t* w_ring = zero_blk + C::kZeroBytes;    // [kWStages][box0 | box1]
     uint64_t* bars = reinterpret_cast<uint64_t*>(w_ring + C::kWBytes);
     uint64_t* w_full = bars;
     uint64_t* w_empty = w_full + C::kWStages;
@@ -138,6 +146,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+    if constexpr (BBULK) {
+        // read by the tensor cores (async proxy) through the MMA descriptors
+        for (uint32_t i = threadIdx.x; i < C::kZeroBytes / 16; i += blockDim.x)
+            reinterpret_cast<uint4*>(zero_blk)[i] = make_uint4(0u, 0u, 0u, 0u);
+        fence_async_smem();
+    }
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::kWStages; ++i) {
             mbar_init(&w_full[i], 1);
@@ -222,7 +236,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
                 int out_rows = 128;
                 const uint16_t* Bbase = nullptr;
                 int out = 0;
-                if (p.b_bulk) {
+                if constexpr (BBULK) {
                     const PairDesc& pd = p.pairs[pair];
                     out = pd.out;
                     Bbase = pd.B;
@@ -235,7 +249,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
                     if (!mbar_wait_bounded(&op_empty[os], oph ^ 1, abort_flag, kWaitLimitNs)) { ok = false; break; }
                     uint8_t* a_dst = op_ring + (size_t)os * C::kOpStageBytes;
                     uint8_t* b_dst = a_dst + C::kABytes;
-                    if (p.b_bulk) {
+                    if constexpr (BBULK) {
                         // rows past the weight's end are not fetched (their
                         // products only reach accumulator rows never stored)
                         const uint32_t bbytes = (uint32_t)out_rows * 16u;
@@ -261,6 +275,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
             constexpr uint32_t idesc = instr_desc_bf16(128, 128, /*B MN-major*/ 1);
+            const uint32_t zero_s = smem_u32(zero_blk);
             int os = 0;
             uint32_t oph = 0, aph = 0;
             for (int64_t t = first; t < p.t_end && !*abort_flag; t += gridDim.x) {
@@ -277,13 +292,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
                     for (int k = 0; k < KP / 16; ++k) {
                         // MMA A operand: B_e slice, 128 x KP, K-major, rows swizzled
                         // rank 8 (bulk-copied, plain core-matrix layout): the
-                        // second 8-deep K chunk re-reads the first (LBO 0); the
-                        // matching A rows 8..15 are TMA zero fill, so it adds 0
-                        const uint64_t da = p.b_bulk
+                        // second 8-deep K chunk re-reads the first (LBO 0) and
+                        // meets the zero A rows below, so it adds 0
+                        const uint64_t da = BBULK
                             ? smem_desc(b_s, 0, 128, kSwizzleNone)
                             : smem_desc(b_s + 32u * k, 16, C::kBSbo, C::kBLayout);
-                        // MMA B operand: A_e slice, KP x 128, N-major, two 64-column halves
-                        const uint64_t db = smem_desc(a_s + 2048u * k, C::kAHalfBytes, 1024, kSwizzle128B);
+                        // MMA B operand: A_e slice, KP x 128, N-major, two 64-column
+                        // halves (LBO apart), 8-row K groups SBO apart.  Rank 8
+                        // holds only K rows 0..7 per half; the K-group stride
+                        // points at the zero block (half 1 lands on its second KB).
+                        const uint64_t db = BBULK
+                            ? smem_desc(a_s, C::kAHalfBytes, zero_s - a_s, kSwizzle128B)
+                            : smem_desc(a_s + 2048u * k, C::kAHalfBytes, 1024, kSwizzle128B);
                         tc_mma_f16(tmem_base + 128u * ei, da, db, idesc, k > 0 ? 1u : 0u);
                     }
                     tc_commit(&op_empty[os]);
