@@ -50,6 +50,8 @@ def parse():
                     help="switch kernel: tensor-core (tc), mma.sync (mma), or auto")
     ap.add_argument("--mode", choices=["switch", "rebase"], default="switch",
                     help="in-place switch (prev -> cur) or re-base from a pristine copy W0")
+    ap.add_argument("--router-tokens", type=int, default=4096,
+                    help="also time the pre-gate alone on this many tokens (0 = skip)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -392,6 +394,36 @@ def run_ours(args):
         e2e = {"value": round(e_units * w_bytes / (e_max / 1000) / 1e9, 2),
                "unit": "GB/s", "h2d_bytes_per_step": cfg.d * 4, "d2h_bytes_per_step": 16}
 
+    # the router alone on a batch of tokens (the Llama-3-8B-shaped router
+    # batch: T=4096, d=4096, E=8): an HBM-bound GEMV over h
+    router = None
+    if args.router_tokens > 0 and rank == 0:
+        Tr = args.router_tokens
+        hr = torch.empty((Tr, cfg.d), dtype=torch.float32, device="cuda")
+        hr.normal_(0.0, 1.0, generator=torch.Generator(device="cuda").manual_seed(cfg.seed() + 17))
+        rr = torch.zeros((Tr, 4), dtype=torch.int32, device="cuda")
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")  # > L2 (126 MB)
+        for _ in range(3):
+            sw.pregate(hr, model.Wr, rr, sh)
+        ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(10)]
+        ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(10)]
+        for i in range(10):
+            flush.zero_()                      # evict h from L2 between timed launches
+            ev0[i].record(stream)
+            sw.pregate(hr, model.Wr, rr, sh)
+            ev1[i].record(stream)
+        torch.cuda.synchronize()
+        rms = [a.elapsed_time(b) for a, b in zip(ev0, ev1)]
+        r_ms = statistics.median(rms)
+        del flush
+        r_bytes = Tr * cfg.d * 4 + cfg.d * cfg.n_experts * 4 + Tr * 16
+        router = {"tokens": Tr, "d": cfg.d, "experts": cfg.n_experts,
+                  "ms_p50": round(r_ms, 5), "tokens_per_s": round(Tr / (r_ms / 1e3)),
+                  "hbm_gbs": round(r_bytes / (r_ms / 1e3) / 1e9, 1),
+                  "frac_of_peak": round(r_bytes / (r_ms / 1e3) / 1e9 / measured_peaks()[0], 4),
+                  "l2": "flushed (256 MB write) before each timed launch"}
+        del hr, rr
+
     peak, peak_kind = measured_peaks()
     sw_avg = statistics.mean(sw_ms)
     achieved = w_bytes / (sw_avg / 1000.0) / 1e9
@@ -433,6 +465,7 @@ def run_ours(args):
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": 2 * args.steps,
+            "router": router,
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)

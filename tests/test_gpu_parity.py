@@ -114,7 +114,8 @@ def all_rows(i, out):
 # pre-gating
 
 @pytest.mark.parametrize("T,d,E", [(1, 4, 1), (1, 4096, 8), (7, 256, 4), (64, 4096, 8),
-                                   (33, 5120, 16), (5, 264, 33), (9, 128, 64), (300, 512, 3)])
+                                   (33, 5120, 16), (5, 264, 33), (9, 128, 64), (300, 512, 3),
+                                   (4096, 4096, 8)])   # the Llama-3-8B-shaped router batch
 def test_pregate_matches_oracle(T, d, E):
     cfg = wl.custom("p", 1, [("q", 8, 8)], n_experts=E, rank=8, alpha=16, n_tokens=T, d=d)
     model = wl.make_model(cfg, device="cuda", seed=11 + E)
