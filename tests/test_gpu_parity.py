@@ -115,7 +115,8 @@ def all_rows(i, out):
 
 @pytest.mark.parametrize("T,d,E", [(1, 4, 1), (1, 4096, 8), (7, 256, 4), (64, 4096, 8),
                                    (33, 5120, 16), (5, 264, 33), (9, 128, 64), (300, 512, 3),
-                                   (4096, 4096, 8)])   # the Llama-3-8B-shaped router batch
+                                   (4096, 4096, 8),    # the Llama-3-8B-shaped router batch
+                                   (512, 1024, 16), (257, 2944, 12)])
 def test_pregate_matches_oracle(T, d, E):
     cfg = wl.custom("p", 1, [("q", 8, 8)], n_experts=E, rank=8, alpha=16, n_tokens=T, d=d)
     model = wl.make_model(cfg, device="cuda", seed=11 + E)
@@ -127,6 +128,27 @@ def test_pregate_matches_oracle(T, d, E):
     assert len(amb) <= max(1, T // 50)
     if E == 1:
         assert np.all(got[:, 1] == -1)
+
+
+@pytest.mark.parametrize("E", [8, 16])
+def test_pregate_route_does_not_depend_on_batch_size(E):
+    """A token's route is bitwise the same whether it is gated alone or inside
+    a large batch (the batched path stages Wr in shared memory, the small one
+    reads it through L1, with the same arithmetic order)."""
+    T, d = 1024, 2048
+    cfg = wl.custom("p", 1, [("q", 8, 8)], n_experts=E, rank=8, alpha=16, n_tokens=T, d=d)
+    sw = make_switcher(wl.make_model(cfg, device="cuda"))
+    g = torch.Generator(device="cuda").manual_seed(77)
+    h = torch.randn((T, d), generator=g, device="cuda")
+    Wr = torch.randn((d, E), generator=g, device="cuda") * 0.05
+    batch = torch.zeros((T, 4), dtype=torch.int32, device="cuda")
+    sw.pregate(h, Wr, batch, stream())
+    single = torch.zeros((T, 4), dtype=torch.int32, device="cuda")
+    for t in range(0, T, 97):
+        sw.pregate(h[t:t + 1], Wr, single[t:t + 1], stream())
+    torch.cuda.synchronize()
+    rows = list(range(0, T, 97))
+    assert torch.equal(batch[rows], single[rows])
 
 
 def test_pregate_duplicate_columns_tie_exactly():

@@ -7,6 +7,7 @@
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <new>
 #include <vector>
 
@@ -396,12 +397,34 @@ int adafuse_pregate(adafuse_ctx* ctx, const float* h, int64_t T, int64_t d, cons
     if (!guard.ok) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int E = ctx->n_experts;
-    if (E <= 8) {
-        constexpr int TPB = 8;
-        pregate_kernel<8, TPB><<<(unsigned)ceil_div(T, TPB), kPregateThreads, 0, s>>>(h, T, d, Wr, E, route);
-    } else if (E <= 16) {
-        constexpr int TPB = 4;
-        pregate_kernel<16, TPB><<<(unsigned)ceil_div(T, TPB), kPregateThreads, 0, s>>>(h, T, d, Wr, E, route);
+    if (E <= 16) {
+        // warp-per-token kernel; Wr staged in shared memory for batches that
+        // amortise it (same arithmetic either way)
+        const int emax = E <= 8 ? 8 : 16;
+        const size_t wr_smem = (size_t)d * (emax + 1) * 4;
+        const bool smem = T >= 256 && wr_smem <= 200 * 1024;
+        if (smem) {
+            const int threads = 512;
+            const int64_t groups = ceil_div(T, emax == 8 ? 2 : 1);
+            const int64_t blocks = std::min<int64_t>(ctx->sm_count, ceil_div(groups, threads / 32));
+            if (emax == 8) {
+                cudaFuncSetAttribute(pregate_warp_kernel<8, 2, true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wr_smem);
+                pregate_warp_kernel<8, 2, true><<<(unsigned)blocks, threads, wr_smem, s>>>(h, T, d, Wr, E, route);
+            } else {
+                cudaFuncSetAttribute(pregate_warp_kernel<16, 1, true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wr_smem);
+                pregate_warp_kernel<16, 1, true><<<(unsigned)blocks, threads, wr_smem, s>>>(h, T, d, Wr, E, route);
+            }
+        } else {
+            const int threads = 256;
+            const int64_t groups = ceil_div(T, emax == 8 ? 2 : 1);
+            const int64_t blocks = ceil_div(groups, threads / 32);
+            if (emax == 8)
+                pregate_warp_kernel<8, 2, false><<<(unsigned)blocks, threads, 0, s>>>(h, T, d, Wr, E, route);
+            else
+                pregate_warp_kernel<16, 1, false><<<(unsigned)blocks, threads, 0, s>>>(h, T, d, Wr, E, route);
+        }
     } else if (E <= 32) {
         constexpr int TPB = 2;
         pregate_kernel<32, TPB><<<(unsigned)ceil_div(T, TPB), kPregateThreads, 0, s>>>(h, T, d, Wr, E, route);
