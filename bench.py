@@ -57,13 +57,21 @@ def parse():
     return ap.parse_args()
 
 
-def kernel_source_hash():
-    """sha256 over the CUDA sources and the ABI header (identifies the kernels
-    an ncu capture was taken on)."""
+# the sources that define each profiled kernel and its launch (tensor maps,
+# grid, shared memory); editing any of them voids that kernel's ncu figures
+KERNEL_SOURCES = {
+    "switch_tc_kernel": ["common.cuh", "sm100_ptx.cuh", "switch_tc.cuh", "adafuse_abi.cu"],
+    "switch_mma_kernel": ["common.cuh", "switch_mma.cuh", "adafuse_abi.cu"],
+}
+
+
+def kernel_source_hash(kernel_name="switch_tc_kernel"):
+    """sha256 over the sources of one kernel and the ABI header (identifies the
+    code an ncu capture was taken on)."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "weight_merge_b200", "csrc")
-    files = sorted(os.path.join(csrc, f) for f in os.listdir(csrc) if f.endswith((".cu", ".cuh")))
+    files = [os.path.join(csrc, f) for f in KERNEL_SOURCES[kernel_name]]
     for f in files + [os.path.join(ROOT, "include", "adafuse.h")]:
         with open(f, "rb") as fh:
             h.update(os.path.basename(f).encode())
@@ -77,7 +85,7 @@ def profiled_traffic(kernel_name, workload):
     d = os.path.join(ROOT, "profiles")
     if not os.path.isdir(d):
         return None
-    want = kernel_source_hash()
+    want = kernel_source_hash(kernel_name)
     for f in sorted(os.listdir(d)):
         if not f.endswith(".md"):
             continue
