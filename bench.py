@@ -60,8 +60,8 @@ def parse():
 # the sources that define each profiled kernel and its launch (tensor maps,
 # grid, shared memory); editing any of them voids that kernel's ncu figures
 KERNEL_SOURCES = {
-    "switch_tc_kernel": ["common.cuh", "sm100_ptx.cuh", "switch_tc.cuh", "adafuse_abi.cu"],
-    "switch_mma_kernel": ["common.cuh", "switch_mma.cuh", "adafuse_abi.cu"],
+    "switch_tc_kernel": ["common.cuh", "sm100_ptx.cuh", "switch_tc.cuh", "switch_tc_host.cuh"],
+    "switch_mma_kernel": ["common.cuh", "switch_mma.cuh"],
 }
 
 

@@ -16,6 +16,7 @@
 #include "pregate.cuh"
 #include "switch_mma.cuh"
 #include "switch_tc.cuh"
+#include "switch_tc_host.cuh"
 
 using namespace adafuse;
 
@@ -106,81 +107,9 @@ int64_t walk_tiles(const adafuse_desc* d, Emit&& emit) {
 
 int kp_class(int r) { return r <= 8 ? 8 : r <= 16 ? 16 : r <= 32 ? 32 : 64; }
 
-// The tensor-core kernel needs TMA-legal strides (rank a multiple of 8).
-int tc_kp_for(int r) { return (r % 8 != 0 || r > 64) ? 0 : r <= 16 ? 16 : r <= 32 ? 32 : 64; }
-
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_tiled_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    }
-    return fn;
-}
-
-// W [out, in]: box 64 x 128 (cols x rows), 128B swizzle.
-// A [E, r, in]: box 64 x KP x 1, 128B swizzle (rows past r read as zero).
-// B [E, out, r]: box KP x 128 x 1, swizzle = KP*2 bytes (cols past r read as zero).
-bool encode_pair_maps(EncodeTiledFn enc, const PairDesc& pd, int E, int r, int kp,
-                      CUtensorMap out[3]) {
-    const cuuint32_t ones[3] = {1, 1, 1};
-    {
-        const cuuint64_t dims[2] = {(cuuint64_t)pd.in, (cuuint64_t)pd.out};
-        const cuuint64_t strides[1] = {(cuuint64_t)pd.in * 2};
-        const cuuint32_t box[2] = {64, 128};
-        if (enc(&out[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (void*)pd.W, dims, strides, box,
-                ones, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return false;
-    }
-    {
-        const cuuint64_t dims[3] = {(cuuint64_t)pd.in, (cuuint64_t)r, (cuuint64_t)E};
-        const cuuint64_t strides[2] = {(cuuint64_t)pd.in * 2, (cuuint64_t)pd.in * r * 2};
-        // rank 8 fetches exactly its 8 rows; other ranks a KP-row box whose
-        // rows past r read as zero
-        const cuuint32_t box[3] = {64, (cuuint32_t)(r == 8 ? 8 : kp), 1};
-        if (enc(&out[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, (void*)pd.A, dims, strides, box,
-                ones, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return false;
-    }
-    {
-        const cuuint64_t dims[3] = {(cuuint64_t)r, (cuuint64_t)pd.out, (cuuint64_t)E};
-        const cuuint64_t strides[2] = {(cuuint64_t)r * 2, (cuuint64_t)pd.out * r * 2};
-        const cuuint32_t box[3] = {(cuuint32_t)kp, 128, 1};
-        const CUtensorMapSwizzle sw = kp == 16 ? CU_TENSOR_MAP_SWIZZLE_32B
-                                    : kp == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
-                                               : CU_TENSOR_MAP_SWIZZLE_128B;
-        if (enc(&out[2], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, (void*)pd.B, dims, strides, box,
-                ones, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return false;
-    }
-    return true;
-}
-
 template <int KP, bool BBULK>
 cudaError_t launch_tc(const adafuse_ctx* c, int64_t t0, int64_t t1, const adafuse_route* prev,
                       const adafuse_route* cur, cudaStream_t s, bool rebase) {
-    const int smem = (int)TcConfig<KP, BBULK>::kSmemBytes;
-    static int configured_for = -1;  // device ordinal the attribute was set on
-    if (configured_for != c->device) {
-        cudaError_t e = cudaFuncSetAttribute(switch_tc_kernel<KP, BBULK>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        configured_for = c->device;
-    }
     TcParams prm;
     prm.pairs = c->d_pairs;
     prm.tiles = c->d_tiles;
@@ -194,10 +123,7 @@ cudaError_t launch_tc(const adafuse_ctx* c, int64_t t0, int64_t t1, const adafus
     prm.status = c->d_status;
     prm.rebase = rebase ? 1 : 0;
     prm.w0_maps = c->d_w0_maps;
-    const int64_t n = t1 - t0;
-    const unsigned grid = (unsigned)(n < c->sm_count ? n : c->sm_count);
-    switch_tc_kernel<KP, BBULK><<<grid, kTcThreads, smem, s>>>(prm);
-    return cudaGetLastError();
+    return launch_switch_tc<KP, BBULK>(prm, c->device, c->sm_count, s);
 }
 
 }  // namespace
@@ -397,40 +323,39 @@ int adafuse_pregate(adafuse_ctx* ctx, const float* h, int64_t T, int64_t d, cons
     if (!guard.ok) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int E = ctx->n_experts;
-    if (E <= 16) {
-        // warp-per-token kernel; Wr staged in shared memory for batches that
-        // amortise it (same arithmetic either way)
-        const int emax = E <= 8 ? 8 : 16;
-        const size_t wr_smem = (size_t)d * (emax + 1) * 4;
-        const bool smem = T >= 256 && wr_smem <= 200 * 1024;
-        if (smem) {
-            const int threads = 512;
-            const int64_t groups = ceil_div(T, emax == 8 ? 2 : 1);
-            const int64_t blocks = std::min<int64_t>(ctx->sm_count, ceil_div(groups, threads / 32));
-            if (emax == 8) {
-                cudaFuncSetAttribute(pregate_warp_kernel<8, 2, true>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wr_smem);
-                pregate_warp_kernel<8, 2, true><<<(unsigned)blocks, threads, wr_smem, s>>>(h, T, d, Wr, E, route);
-            } else {
-                cudaFuncSetAttribute(pregate_warp_kernel<16, 1, true>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wr_smem);
-                pregate_warp_kernel<16, 1, true><<<(unsigned)blocks, threads, wr_smem, s>>>(h, T, d, Wr, E, route);
-            }
-        } else {
-            const int threads = 256;
-            const int64_t groups = ceil_div(T, emax == 8 ? 2 : 1);
-            const int64_t blocks = ceil_div(groups, threads / 32);
-            if (emax == 8)
-                pregate_warp_kernel<8, 2, false><<<(unsigned)blocks, threads, 0, s>>>(h, T, d, Wr, E, route);
-            else
-                pregate_warp_kernel<16, 1, false><<<(unsigned)blocks, threads, 0, s>>>(h, T, d, Wr, E, route);
+    const int emax = E <= 8 ? 8 : E <= 16 ? 16 : E <= 32 ? 32 : 64;
+    const int tpb = 64 / emax;   // tokens per CTA group: TPB x EMAX partial logits per thread
+    const int64_t groups = ceil_div(T, tpb);
+    // Wr in shared memory for batches that amortise staging it (persistent
+    // CTAs); otherwise read from global memory.  Same arithmetic either way.
+    const size_t wr_smem = (size_t)d * (emax + 1) * 4;
+    const bool shared = T >= 256 && wr_smem <= 160 * 1024;
+    const unsigned grid = (unsigned)(shared ? std::min<int64_t>(groups, (int64_t)ctx->sm_count) : groups);
+    auto go = [&](auto kernel, size_t smem) {
+        if (smem > 0) cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        kernel<<<grid, kPregateThreads, smem, s>>>(h, T, d, Wr, E, route);
+    };
+    if (shared) {
+        switch (emax) {
+            case 8: go(pregate_kernel<8, 8, kWrShared>, wr_smem); break;
+            case 16: go(pregate_kernel<16, 4, kWrShared>, wr_smem); break;
+            case 32: go(pregate_kernel<32, 2, kWrShared>, wr_smem); break;
+            default: go(pregate_kernel<64, 1, kWrShared>, wr_smem); break;
         }
-    } else if (E <= 32) {
-        constexpr int TPB = 2;
-        pregate_kernel<32, TPB><<<(unsigned)ceil_div(T, TPB), kPregateThreads, 0, s>>>(h, T, d, Wr, E, route);
+    } else if (E == emax) {
+        switch (emax) {
+            case 8: go(pregate_kernel<8, 8, kWrVector>, 0); break;
+            case 16: go(pregate_kernel<16, 4, kWrVector>, 0); break;
+            case 32: go(pregate_kernel<32, 2, kWrVector>, 0); break;
+            default: go(pregate_kernel<64, 1, kWrVector>, 0); break;
+        }
     } else {
-        constexpr int TPB = 1;
-        pregate_kernel<64, TPB><<<(unsigned)ceil_div(T, TPB), kPregateThreads, 0, s>>>(h, T, d, Wr, E, route);
+        switch (emax) {
+            case 8: go(pregate_kernel<8, 8, kWrScalar>, 0); break;
+            case 16: go(pregate_kernel<16, 4, kWrScalar>, 0); break;
+            case 32: go(pregate_kernel<32, 2, kWrScalar>, 0); break;
+            default: go(pregate_kernel<64, 1, kWrScalar>, 0); break;
+        }
     }
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? ADAFUSE_OK : cuda_fail(e, "pregate launch");

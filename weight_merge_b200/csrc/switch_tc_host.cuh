@@ -1,0 +1,95 @@
+// switch_tc_host.cuh -- host side of the tensor-core switch: which ranks it
+// takes, the TMA tensor maps of each (layer, target) weight, and the launch.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "switch_tc.cuh"
+
+namespace adafuse {
+
+// The tensor-core kernel needs TMA-legal strides (rank a multiple of 8).
+inline int tc_kp_for(int r) { return (r % 8 != 0 || r > 64) ? 0 : r <= 16 ? 16 : r <= 32 ? 32 : 64; }
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_tiled_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+// W [out, in]: box 64 x 128 (cols x rows), 128B swizzle.
+// A [E, r, in]: box 64 x KP x 1, 128B swizzle (rows past r read as zero).
+// B [E, out, r]: box KP x 128 x 1, swizzle = KP*2 bytes (cols past r read as zero).
+inline bool encode_pair_maps(EncodeTiledFn enc, const PairDesc& pd, int E, int r, int kp,
+                      CUtensorMap out[3]) {
+    const cuuint32_t ones[3] = {1, 1, 1};
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)pd.in, (cuuint64_t)pd.out};
+        const cuuint64_t strides[1] = {(cuuint64_t)pd.in * 2};
+        const cuuint32_t box[2] = {64, 128};
+        if (enc(&out[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (void*)pd.W, dims, strides, box,
+                ones, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return false;
+    }
+    {
+        const cuuint64_t dims[3] = {(cuuint64_t)pd.in, (cuuint64_t)r, (cuuint64_t)E};
+        const cuuint64_t strides[2] = {(cuuint64_t)pd.in * 2, (cuuint64_t)pd.in * r * 2};
+        // rank 8 fetches exactly its 8 rows; other ranks a KP-row box whose
+        // rows past r read as zero
+        const cuuint32_t box[3] = {64, (cuuint32_t)(r == 8 ? 8 : kp), 1};
+        if (enc(&out[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, (void*)pd.A, dims, strides, box,
+                ones, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return false;
+    }
+    {
+        const cuuint64_t dims[3] = {(cuuint64_t)r, (cuuint64_t)pd.out, (cuuint64_t)E};
+        const cuuint64_t strides[2] = {(cuuint64_t)r * 2, (cuuint64_t)pd.out * r * 2};
+        const cuuint32_t box[3] = {(cuuint32_t)kp, 128, 1};
+        const CUtensorMapSwizzle sw = kp == 16 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                    : kp == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                               : CU_TENSOR_MAP_SWIZZLE_128B;
+        if (enc(&out[2], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, (void*)pd.B, dims, strides, box,
+                ones, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return false;
+    }
+    return true;
+}
+
+// One launch of the tensor-core switch: persistent grid (one CTA per SM, at
+// most one per tile), dynamic shared memory opted in once per device.
+template <int KP, bool BBULK>
+cudaError_t launch_switch_tc(const TcParams& prm, int device, int sm_count, cudaStream_t s) {
+    const int smem = (int)TcConfig<KP, BBULK>::kSmemBytes;
+    static int configured_for = -1;  // device ordinal the attribute was set on
+    if (configured_for != device) {
+        cudaError_t e = cudaFuncSetAttribute(switch_tc_kernel<KP, BBULK>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        configured_for = device;
+    }
+    const int64_t n = prm.t_end - prm.t_begin;
+    const unsigned grid = (unsigned)(n < sm_count ? n : sm_count);
+    switch_tc_kernel<KP, BBULK><<<grid, kTcThreads, smem, s>>>(prm);
+    return cudaGetLastError();
+}
+
+}  // namespace adafuse
