@@ -54,7 +54,7 @@ struct TcConfig {
     static_assert(KP == 16 || KP == 32 || KP == 64, "KP");
     static_assert(!BBULK || KP == 16, "the bulk path is rank 8");
     static constexpr int kWStages = BBULK ? 6 : KP == 64 ? 3 : KP == 32 ? 4 : 5;
-    static constexpr int kOpStages = KP == 16 ? 6 : KP == 32 ? 4 : 3;
+    static constexpr int kOpStages = KP == 16 ? 6 : 4;
     static constexpr uint32_t kARows = BBULK ? 8 : KP;             // A rows fetched
     static constexpr uint32_t kAHalfBytes = kARows * 128;          // rows x 64 cols bf16
     static constexpr uint32_t kABytes = 2 * kAHalfBytes;
