@@ -1,0 +1,162 @@
+"""GPU edge cases of the switch and the pre-gate, against the fp64 oracle.
+
+Degenerate and extreme inputs the AdaFuse switch (gist.science technical
+summary, section 2-na) must still get right: results in the bf16 subnormal
+range, W values at the edge of overflow, an empty token batch, and the
+pre-gate + switch pair captured into a CUDA graph and replayed.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from weight_merge_b200 import binding as Bnd
+from weight_merge_b200 import workloads as wl
+
+from .util import bits, check_switch_rows, make_routes, route_tuple, routes_to_np
+
+pytestmark = pytest.mark.gpu
+
+MMA, TC = Bnd.ADAFUSE_KERNEL_MMA_SYNC, Bnd.ADAFUSE_KERNEL_TCGEN05
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from weight_merge_b200 import build
+    build.build()
+    oracle.build()
+
+
+def stream():
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _model(kernel, scale_w=1.0, scale_a=1.0, scale_b=1.0, seed=0, r=8):
+    cfg = wl.custom("edge", 2, [("a", 136, 264), ("b", 256, 128)], n_experts=4, rank=r,
+                    alpha=2.0 * r, n_tokens=2, d=264)
+    m = wl.make_model(cfg, device="cuda", seed=seed)
+    with torch.no_grad():
+        for w in m.W:
+            w.copy_((w.float() * scale_w).to(torch.bfloat16))
+        for a in m.A:
+            a.copy_((a.float() * scale_a).to(torch.bfloat16))
+        for b in m.B:
+            b.copy_((b.float() * scale_b).to(torch.bfloat16))
+    sw = Bnd.Switcher(m.W, m.A, m.B, cfg.n_layers, len(cfg.targets), cfg.n_experts, cfg.rank,
+                      cfg.alpha, device=torch.cuda.current_device())
+    sw.set_kernel(kernel)
+    return cfg, m, sw
+
+
+def _switch_and_check(cfg, m, sw, routes, steps):
+    r_np = routes_to_np(routes)
+    A_h = [bits(a) for a in m.A]
+    B_h = [bits(b) for b in m.B]
+    for p, c in steps:
+        before = [bits(w) for w in m.W]
+        sw.switch(None if p is None else Bnd.Switcher.route_ptr(routes, p),
+                  None if c is None else Bnd.Switcher.route_ptr(routes, c), stream())
+        torch.cuda.synchronize()
+        assert sw.status(stream()) == 0
+        for i, w in enumerate(m.W):
+            rows = np.arange(w.shape[0], dtype=np.int64)
+            check_switch_rows(bits(w), before[i], rows, w.shape[0], A_h[i], B_h[i], cfg.scale,
+                              None if p is None else route_tuple(r_np, p),
+                              None if c is None else route_tuple(r_np, c))
+
+
+@pytest.mark.parametrize("kernel", [MMA, TC])
+def test_subnormal_results(kernel):
+    """W ~ 1e-39 and dW of the same size: every result is a bf16 subnormal
+    (below 2^-126), which fp32 arithmetic without flush-to-zero keeps."""
+    # W ~ N(0, .02) * 5e-38 -> ~1e-39; B ~ .01 * 1e-37, A ~ .06 -> B*A ~ 6e-41 per term
+    cfg, m, sw = _model(kernel, scale_w=5e-38, scale_b=1e-37, seed=3)
+    sub = sum(int(((bits(w) & 0x7F80) == 0).sum()) for w in m.W)
+    assert sub > 0.9 * sum(w.numel() for w in m.W)
+    routes = make_routes(np.array([[0, 2], [3, 1]], np.int32),
+                         np.array([[0.7, 0.3], [0.6, 0.4]], np.float32))
+    _switch_and_check(cfg, m, sw, routes, [(None, 0), (0, 1), (1, None)])
+
+
+@pytest.mark.parametrize("kernel", [MMA, TC])
+def test_overflow_to_infinity(kernel):
+    """W at the largest bf16 magnitudes plus a same-signed dW rounds to +-inf,
+    as the oracle's round-to-nearest-even does."""
+    cfg, m, sw = _model(kernel, seed=4)
+    with torch.no_grad():
+        for w in m.W:
+            w.copy_(torch.where(w >= 0, 3.3895e38, -3.3895e38).to(torch.bfloat16))
+        # |B| ~ 2e36, |A| ~ 0.05: dW ~ 1e36 > half a bf16 step at 3.39e38 (6.6e35),
+        # positive everywhere, while every fp32 partial stays finite
+        for b in m.B:
+            b.abs_().mul_(3e38)
+        for a in m.A:
+            a.abs_()
+    routes = make_routes(np.array([[0, 1]], np.int32), np.array([[0.5, 0.5]], np.float32))
+    before = [bits(w) for w in m.W]
+    sw.switch(None, Bnd.Switcher.route_ptr(routes, 0), stream())
+    torch.cuda.synchronize()
+    A_h = [bits(a) for a in m.A]
+    B_h = [bits(b) for b in m.B]
+    r_np = routes_to_np(routes)
+    for i, w in enumerate(m.W):
+        got = bits(w)
+        want = oracle.switch(before[i], A_h[i], B_h[i], cfg.scale, None, route_tuple(r_np, 0))
+        inf_want = (want & 0x7FFF) == 0x7F80
+        assert inf_want.sum() > 0                       # some really overflow
+        assert np.array_equal(got[inf_want], want[inf_want])
+        # negative W moves away from the overflow and stays finite
+        fin = ~inf_want
+        assert np.all((got[fin] & 0x7F80) != 0x7F80)
+
+
+def test_pregate_empty_batch_is_a_noop():
+    cfg, m, sw = _model(TC)
+    h = torch.empty((0, cfg.d), device="cuda")
+    routes = torch.full((1, 4), 7, dtype=torch.int32, device="cuda")
+    sw.pregate(h, m.Wr, routes, stream())
+    torch.cuda.synchronize()
+    assert torch.all(routes == 7)
+
+
+@pytest.mark.parametrize("kernel", [MMA, TC])
+def test_cuda_graph_capture_of_pregate_and_switch(kernel):
+    """One decode step (pre-gate the token, switch prev -> cur, keep cur as the
+    next prev) captured once and replayed gives the same W, bit for bit, as
+    the same calls made eagerly."""
+    cfg, m1, s1 = _model(kernel, seed=9)
+    _, m2, s2 = _model(kernel, seed=9)
+    g = torch.Generator(device="cuda").manual_seed(5)
+    T = 4
+    hs = torch.randn((T, cfg.d), generator=g, device="cuda")
+    # eager
+    r1 = torch.zeros((T, 4), dtype=torch.int32, device="cuda")
+    for t in range(T):
+        s1.pregate(hs[t:t + 1], m1.Wr, r1[t:t + 1], stream())
+        s1.switch(None if t == 0 else Bnd.Switcher.route_ptr(r1, t - 1),
+                  Bnd.Switcher.route_ptr(r1, t), stream())
+    # graph: fixed buffers for the token, the previous and the current route
+    h_slot = torch.empty((1, cfg.d), device="cuda")
+    prev = torch.zeros((1, 4), dtype=torch.int32, device="cuda")
+    cur = torch.zeros((1, 4), dtype=torch.int32, device="cuda")
+    h_slot.copy_(hs[0:1])
+    s2.pregate(h_slot, m2.Wr, cur, stream())          # token 0, eagerly (no prev)
+    s2.switch(None, Bnd.Switcher.route_ptr(cur, 0), stream())
+    prev.copy_(cur)
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            sh = side.cuda_stream
+            s2.pregate(h_slot, m2.Wr, cur, sh)
+            s2.switch(Bnd.Switcher.route_ptr(prev, 0), Bnd.Switcher.route_ptr(cur, 0), sh)
+            prev.copy_(cur)
+    for t in range(1, T):
+        h_slot.copy_(hs[t:t + 1])
+        graph.replay()
+    torch.cuda.synchronize()
+    assert s2.status(stream()) == 0
+    for a, b in zip(m1.W, m2.W):
+        assert torch.equal(a, b)
+    assert torch.equal(r1[T - 1:T], cur)
