@@ -217,6 +217,13 @@ def oracle_rate(cfg, target_s=10.0, seed_layers=1):
     return gbs, oracle.num_threads(), desc, dt, elems
 
 
+def workload_label(cfg, n_tokens):
+    from weight_merge_b200 import workloads as wl
+    return (f"{cfg.name}: {cfg.shape}, {cfg.n_layers} layers x {len(cfg.targets)} targets "
+            f"({wl.describe_targets(cfg)}), E={cfg.n_experts}, r={cfg.rank}, "
+            f"alpha={cfg.alpha:g}, top-2, {n_tokens}-token decode switch sequence")
+
+
 # --------------------------------------------------------------------------
 # the reference arm: the oracle, on the host cores
 
@@ -241,8 +248,8 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1000 * statistics.mean(times), 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{cfg.name}: {cfg.n_layers} layers, d={cfg.d}, "
-                               f"E={cfg.n_experts}, r={cfg.rank}, row sample of one layer"},
+        "config": {"workload": workload_label(cfg, cfg.n_tokens),
+                   "sample": "each step times a row sample of one layer"},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads,
                          "kind": "oracle", "sample": desc},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
@@ -450,11 +457,7 @@ def run_ours(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded random weights and hidden states)",
             "config": {
-                "workload": f"{cfg.name}: Llama-2-7B-shaped, {cfg.n_layers} layers x "
-                            f"{len(cfg.targets)} targets (q,k,v,o {cfg.d}x{cfg.d}; gate,up "
-                            f"{cfg.targets[4].out}x{cfg.d}; down {cfg.d}x{cfg.targets[6].inn}), "
-                            f"E={cfg.n_experts}, r={cfg.rank}, alpha={cfg.alpha:g}, top-2, "
-                            f"{T}-token decode switch sequence",
+                "workload": workload_label(cfg, T),
                 "w_bytes_per_switch": w_bytes,
                 "l2": "inputs larger than L2 (W read+write per switch >> 126 MB), no flush",
                 "parallelism": f"replicas x{world}",

@@ -46,6 +46,7 @@ class Config:
     b_std: float = 0.01
     wr_std: float = 0.05
     index: int = 0
+    shape: str = ""                  # the decoder whose weight shapes these are
 
     @property
     def scale(self) -> float:
@@ -79,16 +80,26 @@ def _llama(d, ffn, kv=None):
 
 CONFIGS = {
     "tiny": Config("tiny", 2, 256, (Target("q_proj", 256, 256), Target("v_proj", 256, 256)),
-                   n_experts=4, rank=4, alpha=8.0, n_tokens=16, index=0),
+                   n_experts=4, rank=4, alpha=8.0, n_tokens=16, index=0, shape="tiny"),
     "7b": Config("7b", 32, 4096, _llama(4096, 11008), n_experts=8, rank=8, alpha=16.0,
-                 n_tokens=64, index=1),
+                 n_tokens=64, index=1, shape="Llama-2-7B-shaped"),
     "7b-r64": Config("7b-r64", 32, 4096, _llama(4096, 11008), n_experts=16, rank=64,
-                     alpha=128.0, n_tokens=64, route_mode="share_one", share_p=0.3, index=2),
+                     alpha=128.0, n_tokens=64, route_mode="share_one", share_p=0.3, index=2,
+                     shape="Llama-2-7B-shaped"),
     "13b": Config("13b", 40, 5120, _llama(5120, 13824), n_experts=8, rank=16, alpha=32.0,
-                  n_tokens=128, repeat_p=0.1, index=3),
+                  n_tokens=128, repeat_p=0.1, index=3, shape="Llama-2-13B-shaped"),
     "l3-8b": Config("l3-8b", 32, 4096, _llama(4096, 14336, kv=1024), n_experts=8, rank=16,
-                    alpha=32.0, n_tokens=256, route_mode="zipf", pregate_T=4096, index=4),
+                    alpha=32.0, n_tokens=256, route_mode="zipf", pregate_T=4096, index=4,
+                    shape="Llama-3-8B-shaped (GQA)"),
 }
+
+
+def describe_targets(cfg: Config) -> str:
+    """'q_proj 4096x4096, ...' with equal shapes grouped: 'q,o 4096x4096; k,v 1024x4096'."""
+    groups = {}
+    for t in cfg.targets:
+        groups.setdefault((t.out, t.inn), []).append(t.name.replace("_proj", ""))
+    return "; ".join(f"{','.join(n)} {o}x{i}" for (o, i), n in groups.items())
 
 
 def scaled(cfg: Config, n_layers: Optional[int] = None, **kw) -> Config:
