@@ -40,14 +40,15 @@ FALLBACK_HBM_GBS = 6650.0
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="7b")
     ap.add_argument("--layers", type=int, default=None,
                     help="override the layer count (small cases for ncu captures)")
-    ap.add_argument("--kernel", choices=["auto", "mma", "tc"], default="auto",
-                    help="switch kernel: tensor-core (tc), mma.sync (mma), or auto")
+    ap.add_argument("--kernel", choices=["auto", "mma", "tc", "tc2"], default="auto",
+                    help="switch kernel: tensor-core (tc), tensor-core on CTA pairs (tc2), "
+                         "mma.sync (mma), or auto")
     ap.add_argument("--mode", choices=["switch", "rebase"], default="switch",
                     help="in-place switch (prev -> cur) or re-base from a pristine copy W0")
     ap.add_argument("--router-tokens", type=int, default=4096,
@@ -62,6 +63,8 @@ def parse():
 KERNEL_SOURCES = {
     "switch_tc_kernel": ["common.cuh", "sm100_ptx.cuh", "switch_tc.cuh", "switch_tc_host.cuh"],
     "switch_mma_kernel": ["common.cuh", "switch_mma.cuh"],
+    "switch_tc2_kernel": ["common.cuh", "sm100_ptx.cuh", "switch_tc.cuh", "switch_tc2.cuh",
+                          "switch_tc_host.cuh"],
 }
 
 
@@ -111,16 +114,45 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def same_gpu_copy_gbs():
+    """Read+write bytes of a 1 GiB bf16 device copy on this GPU, best of 5 (CUDA
+    events): context for the roofline, whose denominator stays the driver's
+    measured peak.  HBM bandwidth differs by several percent between boards."""
+    import torch
+    a = torch.empty(1 << 30, dtype=torch.bfloat16, device="cuda")
+    b = torch.empty_like(a)
+    best = 0.0
+    for i in range(7):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        b.copy_(a)
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= 2:
+            best = max(best, 4.0 * a.numel() / (e0.elapsed_time(e1) * 1e-3) / 1e9)
+    del a, b
+    torch.cuda.empty_cache()
+    return best
+
+
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons sampled during the timed region."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,"
+              "timestamp")
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
         self.path = None
+        self.t0 = self.t1 = None   # wall-clock bounds of the timed region
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
 
     def __enter__(self):
         fd, self.path = tempfile.mkstemp(prefix="clocks", suffix=".csv")
@@ -128,7 +160,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -157,13 +189,29 @@ class ClockSampler:
                 os.unlink(self.path)
             except Exception:
                 pass
+        # keep the samples taken inside the timed region
+        window = "timed region"
+        if self.t0 is not None and self.t1 is not None:
+            import datetime
+            inside = []
+            for r in rows:
+                try:
+                    ts = datetime.datetime.strptime(r[9], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                except Exception:
+                    continue
+                if self.t0 <= ts <= self.t1:
+                    inside.append(r)
+            if inside:
+                rows = inside
+            else:
+                window = "whole run (no sample fell inside the timed region)"
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
         sm = [int(r[1]) for r in rows]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": int(rows[0][2]),
-                "reasons": reasons, "samples": len(rows),
+                "reasons": reasons, "samples": len(rows), "window": window,
                 "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())
                 if any(r[3].replace(".", "").isdigit() for r in rows) else None}
 
@@ -303,9 +351,10 @@ def run_ours(args):
     sw = B.Switcher(model.W, model.A, model.B, cfg.n_layers, len(cfg.targets), cfg.n_experts,
                     cfg.rank, cfg.alpha, device=dev, names=[t.name for t in cfg.targets])
     sw.set_kernel({"auto": B.ADAFUSE_KERNEL_AUTO, "mma": B.ADAFUSE_KERNEL_MMA_SYNC,
-                   "tc": B.ADAFUSE_KERNEL_TCGEN05}[args.kernel])
+                   "tc": B.ADAFUSE_KERNEL_TCGEN05, "tc2": B.ADAFUSE_KERNEL_TCGEN05_PAIR}[args.kernel])
     kernel_name = {B.ADAFUSE_KERNEL_MMA_SYNC: "switch_mma_kernel",
-                   B.ADAFUSE_KERNEL_TCGEN05: "switch_tc_kernel"}[sw.kernel]
+                   B.ADAFUSE_KERNEL_TCGEN05: "switch_tc_kernel",
+                   B.ADAFUSE_KERNEL_TCGEN05_PAIR: "switch_tc2_kernel"}[sw.kernel]
     rebase = args.mode == "rebase"
     if rebase:
         sw.set_base([w.clone() for w in model.W])
@@ -349,6 +398,7 @@ def run_ours(args):
     with ClockSampler(dev) as clk:
         barrier()
         torch.cuda.synchronize()
+        clk.mark_start()
         t_begin.record(stream)
         for k in range(args.steps):
             kk = args.warmup + k
@@ -361,6 +411,7 @@ def run_ours(args):
             prev_t = t
         t_end.record(stream)
         torch.cuda.synchronize()
+        clk.mark_end()
         barrier()
     clocks = clk.summary()
     assert sw.status(sh) == 0
@@ -405,7 +456,14 @@ def run_ours(args):
         torch.cuda.synchronize()
         barrier()
         e_ms = ev0.elapsed_time(ev1)
-        e_max, e_units = reduce_over_ranks(e_ms, args.steps, world, device="cuda")
+        e_real = 0
+        pp = prev_t
+        for k in range(args.steps):
+            t = (args.warmup + args.steps + k) % T
+            if rebase or pp is None or not np.array_equal(r_np[pp], r_np[t]):
+                e_real += 1
+            pp = t
+        e_max, e_units = reduce_over_ranks(e_ms, e_real, world, device="cuda")
         e2e = {"value": round(e_units * w_bytes / (e_max / 1000) / 1e9, 2),
                "unit": "GB/s", "h2d_bytes_per_step": cfg.d * 4, "d2h_bytes_per_step": 16}
 
@@ -449,6 +507,7 @@ def run_ours(args):
                "sample": desc}
 
     if rank == 0:
+        copy_gbs = same_gpu_copy_gbs()
         sw_sorted = sorted(sw_ms)
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
@@ -472,7 +531,9 @@ def run_ours(args):
                          "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "peak_kind": peak_kind,
                          "traffic": profiled_traffic(kernel_name, cfg.name),
-                         "kernel": kernel_name},
+                         "kernel": kernel_name,
+                         "copy_gbs_this_gpu": round(copy_gbs, 1),
+                         "frac_of_this_gpu_copy": round(achieved / copy_gbs, 4)},
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": 2 * args.steps,

@@ -82,9 +82,12 @@ extern "C" {
                                              (the switch is then incomplete) */
 
 /* ---- switch kernel variants (adafuse_set_switch_kernel) ------------------ */
-#define ADAFUSE_KERNEL_AUTO      0  /* tensor-core kernel when the rank allows it, else mma.sync */
+#define ADAFUSE_KERNEL_AUTO      0  /* rank 8: TCGEN05; other multiples of 8: TCGEN05_PAIR;
+                                       any other rank: MMA_SYNC */
 #define ADAFUSE_KERNEL_MMA_SYNC  1  /* register-streaming kernel, any rank in [1, 64] */
 #define ADAFUSE_KERNEL_TCGEN05   2  /* TMA + tcgen05/TMEM kernel, rank a multiple of 8 */
+#define ADAFUSE_KERNEL_TCGEN05_PAIR 3 /* the same on CTA pairs (tcgen05 cta_group::2, 256 x 128
+                                         W blocks), rank a multiple of 8 */
 
 /* One token's routing decision: the two chosen experts and their gates.
  * idx[j] == -1 marks an empty slot (its gate is ignored).  adafuse_pregate
@@ -172,13 +175,14 @@ ADAFUSE_API int adafuse_switch_batch_layers(adafuse_ctx* ctx, int32_t layer_begi
                                 const adafuse_route* cur, void* stream);
 
 /* Choose the kernel adafuse_switch launches for this context (default
- * ADAFUSE_KERNEL_AUTO).  Both compute the same update to within the
- * documented rounding; ADAFUSE_KERNEL_TCGEN05 needs rank % 8 == 0 and
- * returns UNSUPPORTED_SHAPE otherwise.  Host-only, no device work. */
+ * ADAFUSE_KERNEL_AUTO).  All compute the same update to within the
+ * documented rounding; ADAFUSE_KERNEL_TCGEN05 and ADAFUSE_KERNEL_TCGEN05_PAIR
+ * need rank % 8 == 0 and return UNSUPPORTED_SHAPE otherwise.  Host-only, no
+ * device work. */
 ADAFUSE_API int adafuse_set_switch_kernel(adafuse_ctx* ctx, int kernel);
 
-/* The kernel adafuse_switch will launch (ADAFUSE_KERNEL_MMA_SYNC or
- * ADAFUSE_KERNEL_TCGEN05), or a negative code. */
+/* The kernel adafuse_switch will launch (ADAFUSE_KERNEL_MMA_SYNC,
+ * ADAFUSE_KERNEL_TCGEN05 or ADAFUSE_KERNEL_TCGEN05_PAIR), or a negative code. */
 ADAFUSE_API int adafuse_get_switch_kernel(adafuse_ctx* ctx);
 
 /* ---- re-base switch ------------------------------------------------------

@@ -17,7 +17,10 @@ from .util import bits, check_switch_rows, make_routes, route_tuple, routes_to_n
 
 pytestmark = pytest.mark.gpu
 
-MMA, TC = Bnd.ADAFUSE_KERNEL_MMA_SYNC, Bnd.ADAFUSE_KERNEL_TCGEN05
+MMA, TC, TC2 = (Bnd.ADAFUSE_KERNEL_MMA_SYNC, Bnd.ADAFUSE_KERNEL_TCGEN05,
+                Bnd.ADAFUSE_KERNEL_TCGEN05_PAIR)
+# each kernel at a rank it takes
+KERNEL_RANKS = [(MMA, 8), (TC, 8), (TC2, 16)]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -65,12 +68,12 @@ def _switch_and_check(cfg, m, sw, routes, steps):
                               None if c is None else route_tuple(r_np, c))
 
 
-@pytest.mark.parametrize("kernel", [MMA, TC])
-def test_subnormal_results(kernel):
+@pytest.mark.parametrize("kernel,r", KERNEL_RANKS)
+def test_subnormal_results(kernel, r):
     """W ~ 1e-39 and dW of the same size: every result is a bf16 subnormal
     (below 2^-126), which fp32 arithmetic without flush-to-zero keeps."""
     # W ~ N(0, .02) * 5e-38 -> ~1e-39; B ~ .01 * 1e-37, A ~ .06 -> B*A ~ 6e-41 per term
-    cfg, m, sw = _model(kernel, scale_w=5e-38, scale_b=1e-37, seed=3)
+    cfg, m, sw = _model(kernel, scale_w=5e-38, scale_b=1e-37, seed=3, r=r)
     sub = sum(int(((bits(w) & 0x7F80) == 0).sum()) for w in m.W)
     assert sub > 0.9 * sum(w.numel() for w in m.W)
     routes = make_routes(np.array([[0, 2], [3, 1]], np.int32),
@@ -78,11 +81,11 @@ def test_subnormal_results(kernel):
     _switch_and_check(cfg, m, sw, routes, [(None, 0), (0, 1), (1, None)])
 
 
-@pytest.mark.parametrize("kernel", [MMA, TC])
-def test_overflow_to_infinity(kernel):
+@pytest.mark.parametrize("kernel,r", KERNEL_RANKS)
+def test_overflow_to_infinity(kernel, r):
     """W at the largest bf16 magnitudes plus a same-signed dW rounds to +-inf,
     as the oracle's round-to-nearest-even does."""
-    cfg, m, sw = _model(kernel, seed=4)
+    cfg, m, sw = _model(kernel, seed=4, r=r)
     with torch.no_grad():
         for w in m.W:
             w.copy_(torch.where(w >= 0, 3.3895e38, -3.3895e38).to(torch.bfloat16))
@@ -119,13 +122,13 @@ def test_pregate_empty_batch_is_a_noop():
     assert torch.all(routes == 7)
 
 
-@pytest.mark.parametrize("kernel", [MMA, TC])
-def test_cuda_graph_capture_of_pregate_and_switch(kernel):
+@pytest.mark.parametrize("kernel,r", KERNEL_RANKS)
+def test_cuda_graph_capture_of_pregate_and_switch(kernel, r):
     """One decode step (pre-gate the token, switch prev -> cur, keep cur as the
     next prev) captured once and replayed gives the same W, bit for bit, as
     the same calls made eagerly."""
-    cfg, m1, s1 = _model(kernel, seed=9)
-    _, m2, s2 = _model(kernel, seed=9)
+    cfg, m1, s1 = _model(kernel, seed=9, r=r)
+    _, m2, s2 = _model(kernel, seed=9, r=r)
     g = torch.Generator(device="cuda").manual_seed(5)
     T = 4
     hs = torch.randn((T, cfg.d), generator=g, device="cuda")

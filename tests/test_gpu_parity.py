@@ -38,7 +38,8 @@ def stream():
     return torch.cuda.current_stream().cuda_stream
 
 
-MMA, TC = Bnd.ADAFUSE_KERNEL_MMA_SYNC, Bnd.ADAFUSE_KERNEL_TCGEN05
+MMA, TC, TC2 = (Bnd.ADAFUSE_KERNEL_MMA_SYNC, Bnd.ADAFUSE_KERNEL_TCGEN05,
+                Bnd.ADAFUSE_KERNEL_TCGEN05_PAIR)
 
 
 def make_switcher(model: wl.Model, kernel: int = Bnd.ADAFUSE_KERNEL_AUTO) -> Bnd.Switcher:
@@ -53,7 +54,13 @@ def make_switcher(model: wl.Model, kernel: int = Bnd.ADAFUSE_KERNEL_AUTO) -> Bnd
 
 
 def kernels_for(rank):
-    return [MMA, TC] if rank % 8 == 0 else [MMA]
+    if rank % 8 != 0:
+        return [MMA]
+    return [MMA, TC] if rank == 8 else [MMA, TC, TC2]
+
+
+# (kernel, rank) for the small-model tests: each kernel at a rank it takes
+KERNEL_RANKS = [(MMA, 8), (TC, 8), (TC2, 16)]
 
 
 def host_ab(model):
@@ -216,9 +223,9 @@ def _small_model(seed=3, E=4, r=8):
     return wl.make_model(cfg, device="cuda", seed=seed)
 
 
-@pytest.mark.parametrize("kernel", [MMA, TC])
-def test_identity_switches_leave_w_bit_identical(kernel):
-    model = _small_model()
+@pytest.mark.parametrize("kernel,r", KERNEL_RANKS)
+def test_identity_switches_leave_w_bit_identical(kernel, r):
+    model = _small_model(r=r)
     sw = make_switcher(model, kernel)
     W0 = [bits(w) for w in model.W]
     idx = np.array([[1, 2], [2, 1], [0, 3]], dtype=np.int32)
@@ -233,9 +240,9 @@ def test_identity_switches_leave_w_bit_identical(kernel):
         assert np.array_equal(bits(w), w0)
 
 
-@pytest.mark.parametrize("kernel", [MMA, TC])
-def test_merge_then_unmerge_restores_within_rounding(kernel):
-    model = _small_model(seed=4)
+@pytest.mark.parametrize("kernel,r", KERNEL_RANKS)
+def test_merge_then_unmerge_restores_within_rounding(kernel, r):
+    model = _small_model(seed=4, r=r)
     sw = make_switcher(model, kernel)
     W0 = [bits(w) for w in model.W]
     routes = make_routes(np.array([[0, 3]], np.int32), np.array([[0.55, 0.45]], np.float32))
@@ -253,9 +260,9 @@ def test_merge_then_unmerge_restores_within_rounding(kernel):
         assert np.all(np.abs(f(w2) - f(w0)) <= 0.5 * e(w1) + 0.5 * e(w2) + 1e-30)
 
 
-@pytest.mark.parametrize("kernel", [MMA, TC])
-def test_layer_ranges_equal_one_full_switch(kernel):
-    m1, m2 = _small_model(seed=9), _small_model(seed=9)
+@pytest.mark.parametrize("kernel,r", KERNEL_RANKS)
+def test_layer_ranges_equal_one_full_switch(kernel, r):
+    m1, m2 = _small_model(seed=9, r=r), _small_model(seed=9, r=r)
     s1, s2 = make_switcher(m1, kernel), make_switcher(m2, kernel)
     routes = make_routes(np.array([[0, 1], [2, 3]], np.int32),
                          np.array([[0.7, 0.3], [0.6, 0.4]], np.float32))
@@ -271,10 +278,10 @@ def test_layer_ranges_equal_one_full_switch(kernel):
         s2.switch_layers(2, 2, p(0), p(1), stream())
 
 
-@pytest.mark.parametrize("kernel", [MMA, TC])
+@pytest.mark.parametrize("kernel,r", KERNEL_RANKS)
 @pytest.mark.parametrize("bad", ["index_high", "index_low", "gate_nan", "gate_inf"])
-def test_bad_route_sets_status_and_writes_nothing(bad, kernel):
-    model = _small_model(seed=5)
+def test_bad_route_sets_status_and_writes_nothing(bad, kernel, r):
+    model = _small_model(seed=5, r=r)
     sw = make_switcher(model, kernel)
     W0 = [bits(w) for w in model.W]
     idx = np.array([[0, 1], [2, 3]], np.int32)
@@ -297,9 +304,9 @@ def test_bad_route_sets_status_and_writes_nothing(bad, kernel):
         assert np.array_equal(bits(w), w0)
 
 
-@pytest.mark.parametrize("kernel", [MMA, TC])
-def test_gate_on_empty_slot_is_ignored(kernel):
-    model = _small_model(seed=6)
+@pytest.mark.parametrize("kernel,r", KERNEL_RANKS)
+def test_gate_on_empty_slot_is_ignored(kernel, r):
+    model = _small_model(seed=6, r=r)
     sw = make_switcher(model, kernel)
     routes = make_routes(np.array([[1, -1]], np.int32), np.array([[1.0, np.nan]], np.float32))
     W0 = [bits(w) for w in model.W]
@@ -332,7 +339,7 @@ def _full_size_case(name, n_switches, full_first=True, kernel=Bnd.ADAFUSE_KERNEL
     torch.cuda.empty_cache()
     model = wl.make_model(cfg, device="cuda")
     sw = make_switcher(model, kernel)
-    assert sw.kernel == TC         # the benchmark's launch configuration
+    assert sw.kernel in (TC, TC2)  # a tensor-core kernel, as the benchmark launches
     A_h, B_h = host_ab(model)
     if cfg.route_mode == "router":
         h = wl.make_hidden(cfg, T=n_switches, device="cuda")
@@ -354,25 +361,30 @@ def _full_size_case(name, n_switches, full_first=True, kernel=Bnd.ADAFUSE_KERNEL
 
 
 def test_auto_picks_tensor_cores_when_rank_allows():
-    for r, want in [(4, MMA), (8, TC), (12, MMA), (16, TC), (64, TC)]:
+    for r, want in [(4, MMA), (8, TC), (12, MMA), (16, TC2), (24, TC2), (64, TC2)]:
         cfg = wl.custom("k", 1, [("q", 64, 64)], n_experts=2, rank=r, alpha=2.0 * r, n_tokens=1)
         sw = make_switcher(wl.make_model(cfg, device="cuda"))
         assert sw.kernel == want
         if want == MMA:
             with pytest.raises(Bnd.AdafuseError):
                 sw.set_kernel(TC)
+        if r == 8:
+            with pytest.raises(Bnd.AdafuseError):
+                sw.set_kernel(TC2)
 
 
 def test_llama2_7b_shape_sampled():
     _full_size_case("7b", 3)
 
 
-def test_llama2_7b_r64_shape_sampled():
-    _full_size_case("7b-r64", 3, full_first=False)
+@pytest.mark.parametrize("kernel", [Bnd.ADAFUSE_KERNEL_AUTO, TC, TC2])
+def test_llama2_7b_r64_shape_sampled(kernel):
+    _full_size_case("7b-r64", 3, full_first=False, kernel=kernel)
 
 
-def test_llama2_13b_shape_sampled():
-    _full_size_case("13b", 2, full_first=False)
+@pytest.mark.parametrize("kernel", [Bnd.ADAFUSE_KERNEL_AUTO, TC2])
+def test_llama2_13b_shape_sampled(kernel):
+    _full_size_case("13b", 2, full_first=False, kernel=kernel)
 
 
 def test_llama3_8b_gqa_shape_sampled():

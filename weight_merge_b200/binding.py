@@ -27,6 +27,7 @@ ADAFUSE_STATUS_TIMEOUT = 0x4
 ADAFUSE_KERNEL_AUTO = 0
 ADAFUSE_KERNEL_MMA_SYNC = 1
 ADAFUSE_KERNEL_TCGEN05 = 2
+ADAFUSE_KERNEL_TCGEN05_PAIR = 3
 
 
 class AdafuseError(RuntimeError):

@@ -36,6 +36,10 @@ struct adafuse_ctx {
     std::vector<PairDesc> h_pairs;  // host copy of d_pairs (re-base pointers are patched in)
     CUtensorMap* d_w0_maps = nullptr;  // 1 per pair on the re-base source W0
     bool has_base = false;
+    // pair kernel: 256 x 128 blocks, layer-major like the tile table
+    TileEntry* d_blocks = nullptr;
+    std::vector<int64_t> layer_block_begin;  // [n_layers + 1]
+    int pair_clusters = 0;                   // co-resident CTA pairs (0 = not queried yet)
 };
 
 namespace {
@@ -105,6 +109,25 @@ int64_t walk_tiles(const adafuse_desc* d, Emit&& emit) {
     return n;
 }
 
+// The pair kernel's table: every (layer, target) weight cut into 256 x 128
+// blocks (two 128-row tiles, one per CTA of a pair), in the same order.
+template <typename Emit>
+int64_t walk_blocks(const adafuse_desc* d, Emit&& emit) {
+    int64_t n = 0;
+    for (int32_t l = 0; l < d->n_layers; ++l)
+        for (int32_t k = 0; k < d->n_targets; ++k) {
+            const adafuse_target& t = d->targets[(int64_t)l * d->n_targets + k];
+            const int64_t rb = ceil_div(t.out, kBlockRows), ct = ceil_div(t.in, kTile);
+            for (int64_t i = 0; i < rb; ++i)
+                for (int64_t j = 0; j < ct; ++j) emit(l, k, i, j, n++);
+        }
+    return n;
+}
+
+// The pair kernel takes the tensor-core kernel's ranks except 8 (whose A
+// tensor maps fetch exactly 8 rows for the single-CTA kernel's layout).
+bool pair_eligible(const adafuse_ctx* c) { return c->tc_kp != 0 && c->rank != 8; }
+
 int kp_class(int r) { return r <= 8 ? 8 : r <= 16 ? 16 : r <= 32 ? 32 : 64; }
 
 template <int KP, bool BBULK>
@@ -124,6 +147,32 @@ cudaError_t launch_tc(const adafuse_ctx* c, int64_t t0, int64_t t1, const adafus
     prm.rebase = rebase ? 1 : 0;
     prm.w0_maps = c->d_w0_maps;
     return launch_switch_tc<KP, BBULK>(prm, c->device, c->sm_count, s);
+}
+
+template <int KP>
+cudaError_t launch_tc2(adafuse_ctx* c, int64_t b0, int64_t b1, const adafuse_route* prev,
+                       const adafuse_route* cur, cudaStream_t s, bool rebase) {
+    if (c->pair_clusters == 0) {
+        const cudaError_t e = pair_kernel_clusters<KP>(c->sm_count, &c->pair_clusters);
+        if (e != cudaSuccess) {
+            c->pair_clusters = 0;
+            return e;
+        }
+    }
+    TcParams prm;
+    prm.pairs = c->d_pairs;
+    prm.tiles = c->d_blocks;
+    prm.maps = c->d_maps;
+    prm.t_begin = b0;
+    prm.t_end = b1;
+    prm.prev = prev;
+    prm.cur = cur;
+    prm.E = c->n_experts;
+    prm.s = c->scale;
+    prm.status = c->d_status;
+    prm.rebase = rebase ? 1 : 0;
+    prm.w0_maps = c->d_w0_maps;
+    return launch_switch_tc2<KP>(prm, c->pair_clusters, s);
 }
 
 }  // namespace
@@ -236,6 +285,7 @@ int adafuse_create(adafuse_ctx** out, const adafuse_desc* desc, int device) {
         cudaFree(c->d_tiles);
         cudaFree(c->d_status);
         cudaFree(c->d_maps);
+        cudaFree(c->d_blocks);
         delete c;
         return err == cudaErrorMemoryAllocation ? ADAFUSE_ERR_OUT_OF_MEMORY : cuda_fail(err, what);
     };
@@ -279,6 +329,30 @@ int adafuse_create(adafuse_ctx** out, const adafuse_desc* desc, int device) {
             c->tc_kp = 0;  // fall back to the mma.sync kernel for this context
         }
     }
+    if (pair_eligible(c)) {
+        std::vector<TileEntry> blocks;
+        try {
+            c->layer_block_begin.assign((size_t)desc->n_layers + 1, 0);
+            blocks.reserve((size_t)walk_blocks(desc, [](int, int, int64_t, int64_t, int64_t) {}));
+            walk_blocks(desc, [&](int l, int k, int64_t i, int64_t j, int64_t) {
+                const adafuse_target& tg = desc->targets[(int64_t)l * desc->n_targets + k];
+                TileEntry te;
+                te.x = (uint32_t)((int64_t)l * desc->n_targets + k);
+                if (j * kTile + 64 < tg.in) te.x |= kTileWideBit;
+                if (i * kBlockRows + kTile < tg.out) te.x |= kTileLowerBit;
+                te.y = (uint32_t)((i << 16) | j);
+                blocks.push_back(te);
+                c->layer_block_begin[(size_t)l + 1] = (int64_t)blocks.size();
+            });
+        } catch (...) {
+            return fail(cudaErrorMemoryAllocation, "block table");
+        }
+        if ((e = cudaMalloc(&c->d_blocks, sizeof(TileEntry) * blocks.size())) != cudaSuccess)
+            return fail(e, "cudaMalloc(blocks)");
+        if ((e = cudaMemcpy(c->d_blocks, blocks.data(), sizeof(TileEntry) * blocks.size(),
+                            cudaMemcpyHostToDevice)) != cudaSuccess)
+            return fail(e, "cudaMemcpy(blocks)");
+    }
     *out = c;
     return ADAFUSE_OK;
 }
@@ -291,6 +365,7 @@ int adafuse_destroy(adafuse_ctx* ctx) {
     cudaFree(ctx->d_status);
     cudaFree(ctx->d_maps);
     cudaFree(ctx->d_w0_maps);
+    cudaFree(ctx->d_blocks);
     delete ctx;
     return ADAFUSE_OK;
 }
@@ -298,17 +373,24 @@ int adafuse_destroy(adafuse_ctx* ctx) {
 int adafuse_set_switch_kernel(adafuse_ctx* ctx, int kernel) {
     if (ctx == nullptr) return ADAFUSE_ERR_INVALID_ARG;
     if (kernel != ADAFUSE_KERNEL_AUTO && kernel != ADAFUSE_KERNEL_MMA_SYNC &&
-        kernel != ADAFUSE_KERNEL_TCGEN05)
+        kernel != ADAFUSE_KERNEL_TCGEN05 && kernel != ADAFUSE_KERNEL_TCGEN05_PAIR)
         return ADAFUSE_ERR_INVALID_ARG;
     if (kernel == ADAFUSE_KERNEL_TCGEN05 && ctx->tc_kp == 0) return ADAFUSE_ERR_UNSUPPORTED_SHAPE;
+    if (kernel == ADAFUSE_KERNEL_TCGEN05_PAIR && !pair_eligible(ctx))
+        return ADAFUSE_ERR_UNSUPPORTED_SHAPE;
     ctx->kernel = kernel;
     return ADAFUSE_OK;
 }
 
 int adafuse_get_switch_kernel(adafuse_ctx* ctx) {
     if (ctx == nullptr) return ADAFUSE_ERR_INVALID_ARG;
-    if (ctx->kernel == ADAFUSE_KERNEL_AUTO)
+    if (ctx->kernel == ADAFUSE_KERNEL_AUTO) {
+        // measured on B200 at the Llama shapes: the pair kernel is level at
+        // rank 64 and ahead at rank 16; rank 8 keeps the single-CTA kernel's
+        // bulk-copied B rows and deeper W ring
+        if (pair_eligible(ctx)) return ADAFUSE_KERNEL_TCGEN05_PAIR;
         return ctx->tc_kp != 0 ? ADAFUSE_KERNEL_TCGEN05 : ADAFUSE_KERNEL_MMA_SYNC;
+    }
     return ctx->kernel;
 }
 
@@ -379,7 +461,20 @@ int launch_switch(adafuse_ctx* ctx, int32_t layer_begin, int32_t n_layers,
     DeviceGuard guard(ctx->device);
     if (!guard.ok) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (adafuse_get_switch_kernel(ctx) == ADAFUSE_KERNEL_TCGEN05) {
+    const int kind = adafuse_get_switch_kernel(ctx);
+    if (kind == ADAFUSE_KERNEL_TCGEN05_PAIR) {
+        const int64_t b0 = ctx->layer_block_begin[(size_t)layer_begin];
+        const int64_t b1 = ctx->layer_block_begin[(size_t)layer_begin + n_layers];
+        cudaError_t e = cudaSuccess;
+        if (ctx->tc_kp == 16)
+            e = launch_tc2<16>(ctx, b0, b1, prev, cur, s, rebase);
+        else if (ctx->tc_kp == 32)
+            e = launch_tc2<32>(ctx, b0, b1, prev, cur, s, rebase);
+        else
+            e = launch_tc2<64>(ctx, b0, b1, prev, cur, s, rebase);
+        return e == cudaSuccess ? ADAFUSE_OK : cuda_fail(e, "switch launch");
+    }
+    if (kind == ADAFUSE_KERNEL_TCGEN05) {
         cudaError_t e = cudaSuccess;
         if (ctx->rank == 8)
             e = launch_tc<16, true>(ctx, t0, t1, prev, cur, s, rebase);

@@ -113,6 +113,49 @@ __device__ __forceinline__ TileInfo decode_tile(TileEntry te) {
     return ti;
 }
 
+// Epilogue arithmetic shared by both tensor-core kernels, for one thread's row
+// and 32-column group.
+//   tot = sum_e c_e * acc_e   (experts in order, fused multiply-add in fp32)
+__device__ __forceinline__ void epi_combine(uint32_t t_lane, const Coefs& cf, float (&tot)[32]) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) tot[i] = 0.f;
+#pragma unroll
+    for (int ei = 0; ei < 4; ++ei) {
+        if (ei < cf.n) {
+            const float c = cf.c[ei];
+            float v[32];
+            sm100::tmem_ld32(t_lane + 128u * ei, v);
+            sm100::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) tot[i] = __fmaf_rn(c, v[i], tot[i]);
+        }
+    }
+}
+
+//   W <- bf16_rne(W + tot) for this thread's 32 columns of a 128B-swizzled row
+//   of 64 columns (4 chunks of 16 bytes, chunk index XOR row % 8)
+__device__ __forceinline__ void epi_update_row(uint8_t* rowp, int cgrp, int row, const float (&tot)[32]) {
+    uint4 w[4];
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4) {
+        const int chunk = (cgrp & 1) * 4 + c4;
+        w[c4] = sm100::lds128(rowp + ((chunk ^ (row & 7)) << 4));
+    }
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4) {
+        uint32_t wv[4] = {w[c4].x, w[c4].y, w[c4].z, w[c4].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float lo = __uint_as_float(wv[j] << 16) + tot[8 * c4 + 2 * j];
+            const float hi = __uint_as_float(wv[j] & 0xffff0000u) + tot[8 * c4 + 2 * j + 1];
+            const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+            wv[j] = *reinterpret_cast<const uint32_t*>(&b);
+        }
+        const int chunk = (cgrp & 1) * 4 + c4;
+        sm100::sts128(rowp + ((chunk ^ (row & 7)) << 4), make_uint4(wv[0], wv[1], wv[2], wv[3]));
+    }
+}
+
 template <int KP, bool BBULK>
 __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams p) {
     using C = TcConfig<KP, BBULK>;
@@ -360,19 +403,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
                 aph ^= 1;
                 tc_fence_after();
                 float tot[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) tot[i] = 0.f;
-#pragma unroll
-                for (int ei = 0; ei < 4; ++ei) {
-                    if (ei < cf.n) {
-                        const float c = cf.c[ei];
-                        float v[32];
-                        tmem_ld32(t_lane + 128u * ei, v);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) tot[i] = __fmaf_rn(c, v[i], tot[i]);
-                    }
-                }
+                epi_combine(t_lane, cf, tot);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(acc_empty);
@@ -381,25 +412,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
                 ok = mbar_wait_bounded(&w_full[ws], wph, abort_flag, kWaitLimitNs);
                 if (!__all_sync(0xffffffffu, ok)) { fail(6); break; }
                 uint8_t* rowp = w_ring + (size_t)ws * kWTileBytes + (size_t)half * kWBoxBytes + row * 128;
-                uint4 w[4];
-#pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
-                    const int chunk = (cgrp & 1) * 4 + c4;   // 16-byte chunk within the 128-byte row
-                    w[c4] = lds128(rowp + ((chunk ^ (row & 7)) << 4));
-                }
-#pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
-                    uint32_t wv[4] = {w[c4].x, w[c4].y, w[c4].z, w[c4].w};
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const float lo = __uint_as_float(wv[j] << 16) + tot[8 * c4 + 2 * j];
-                        const float hi = __uint_as_float(wv[j] & 0xffff0000u) + tot[8 * c4 + 2 * j + 1];
-                        const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
-                        wv[j] = *reinterpret_cast<const uint32_t*>(&b);
-                    }
-                    const int chunk = (cgrp & 1) * 4 + c4;
-                    sts128(rowp + ((chunk ^ (row & 7)) << 4), make_uint4(wv[0], wv[1], wv[2], wv[3]));
-                }
+                epi_update_row(rowp, cgrp, row, tot);
                 fence_async_smem();
                 mbar_arrive(&epi_done[ws]);
                 if (++ws == C::kWStages) { ws = 0; wph ^= 1; }

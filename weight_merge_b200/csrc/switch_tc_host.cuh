@@ -7,6 +7,7 @@
 
 #include "common.cuh"
 #include "switch_tc.cuh"
+#include "switch_tc2.cuh"
 
 namespace adafuse {
 
@@ -90,6 +91,54 @@ cudaError_t launch_switch_tc(const TcParams& prm, int device, int sm_count, cuda
     const unsigned grid = (unsigned)(n < sm_count ? n : sm_count);
     switch_tc_kernel<KP, BBULK><<<grid, kTcThreads, smem, s>>>(prm);
     return cudaGetLastError();
+}
+
+// Co-resident CTA pairs of the pair kernel on this device (a persistent grid
+// must not exceed it, or the clusters that do not fit run after the others).
+template <int KP>
+cudaError_t pair_kernel_clusters(int sm_count, int* clusters) {
+    const int smem = (int)Tc2Config<KP>::kSmemBytes;
+    cudaError_t e = cudaFuncSetAttribute(switch_tc2_kernel<KP>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3((unsigned)(sm_count & ~1));
+    cfg.blockDim = dim3(kTcThreads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    e = cudaOccupancyMaxActiveClusters(&n, switch_tc2_kernel<KP>, &cfg);
+    if (e != cudaSuccess) return e;
+    *clusters = n;
+    return n > 0 ? cudaSuccess : cudaErrorInvalidConfiguration;
+}
+
+// One launch of the pair kernel: `clusters` CTA pairs (at most one per block
+// of the table), each persistent over a strided share of the blocks.
+template <int KP>
+cudaError_t launch_switch_tc2(const TcParams& prm, int clusters, cudaStream_t s) {
+    const int smem = (int)Tc2Config<KP>::kSmemBytes;
+    const int64_t n = prm.t_end - prm.t_begin;
+    const int64_t nc = n < clusters ? n : clusters;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3((unsigned)(2 * nc));
+    cfg.blockDim = dim3(kTcThreads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, switch_tc2_kernel<KP>, prm);
 }
 
 }  // namespace adafuse
