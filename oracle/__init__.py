@@ -58,6 +58,9 @@ def _load():
         lib.orc_pregate.argtypes = [P, i64, i64, P, i32, P, P, P]
         lib.orc_switch_rows.argtypes = [P, P, i64, i64, i64, P, P, i32, dbl,
                                         P, P, P, P, P, P]
+        lib.orc_switch_rows_k.argtypes = [P, P, i64, i64, i64, P, P, i32, dbl, i32,
+                                          P, P, P, P, P, P]
+        lib.orc_pregate_topk.argtypes = [P, i64, i64, P, i32, i32, P, P, P]
         lib.orc_num_threads.restype = ctypes.c_int
         lib.orc_set_num_threads.argtypes = [ctypes.c_int]
         _lib = lib
@@ -110,12 +113,40 @@ def pregate(h: np.ndarray, Wr: np.ndarray, return_logits: bool = False):
     return idx, gate
 
 
-def _route_arrays(route):
+def pregate_topk(h: np.ndarray, Wr: np.ndarray, k: int, return_logits: bool = False):
+    """Token-level top-k pre-gating, k in [1, 4] (the pages' router is k = 2).
+
+    h [T, d] fp32, Wr [d, E] fp32  ->  idx [T, k] int32, gate [T, k] fp32
+    (slots past E: idx -1, gate 0), and the fp64 logits when ``return_logits``.
+    """
+    assert 1 <= k <= 4
+    h = np.ascontiguousarray(h, dtype=np.float32)
+    Wr = np.ascontiguousarray(Wr, dtype=np.float32)
+    T, d = h.shape
+    d2, E = Wr.shape
+    assert d == d2
+    idx = np.empty((T, k), dtype=np.int32)
+    gate = np.empty((T, k), dtype=np.float32)
+    z = np.empty((T, E), dtype=np.float64)
+    _load().orc_pregate_topk(_ptr(h), T, d, _ptr(Wr), E, k, _ptr(idx), _ptr(gate), _ptr(z))
+    if return_logits:
+        return idx, gate, z
+    return idx, gate
+
+
+def _route_arrays(route, slots):
     if route is None:
         return None, None
     idx, gate = route
-    return (np.ascontiguousarray(idx, dtype=np.int32).reshape(2),
-            np.ascontiguousarray(gate, dtype=np.float32).reshape(2))
+    return (np.ascontiguousarray(idx, dtype=np.int32).reshape(slots),
+            np.ascontiguousarray(gate, dtype=np.float32).reshape(slots))
+
+
+def _slots(prev, cur):
+    for rt in (prev, cur):
+        if rt is not None:
+            return int(np.asarray(rt[0]).size)
+    return 2
 
 
 def switch_rows(W_rows, row_ids, out: int, A, B, s: float, prev, cur,
@@ -124,7 +155,7 @@ def switch_rows(W_rows, row_ids, out: int, A, B, s: float, prev, cur,
 
     W_rows [n, in] uint16 (bf16 bits), row_ids [n] int64,
     A [E, r, in] uint16, B [E, out, r] uint16,
-    prev / cur: (idx[2], gate[2]) or None.
+    prev / cur: (idx[k], gate[k]) or None, k in [1, 4] (2 for the top-2 router).
     Returns W_new [n, in] uint16, and W + dW in fp64 when ``exact``.
     """
     W_rows = np.ascontiguousarray(W_rows, dtype=np.uint16)
@@ -134,13 +165,20 @@ def switch_rows(W_rows, row_ids, out: int, A, B, s: float, prev, cur,
     B = np.ascontiguousarray(B, dtype=np.uint16)
     E, r, in2 = A.shape
     assert in2 == inn and B.shape == (E, out, r)
-    pi, pg = _route_arrays(prev)
-    ci, cg = _route_arrays(cur)
+    k = _slots(prev, cur)
+    assert 1 <= k <= 4
+    pi, pg = _route_arrays(prev, k)
+    ci, cg = _route_arrays(cur, k)
     W_new = np.empty_like(W_rows)
     W_ex = np.empty((n, inn), dtype=np.float64) if exact else None
-    _load().orc_switch_rows(_ptr(W_rows), _ptr(row_ids), n, out, inn, _ptr(A), _ptr(B),
-                            r, float(s), _ptr(pi), _ptr(pg), _ptr(ci), _ptr(cg),
-                            _ptr(W_new), _ptr(W_ex))
+    if k == 2:
+        _load().orc_switch_rows(_ptr(W_rows), _ptr(row_ids), n, out, inn, _ptr(A), _ptr(B),
+                                r, float(s), _ptr(pi), _ptr(pg), _ptr(ci), _ptr(cg),
+                                _ptr(W_new), _ptr(W_ex))
+    else:
+        _load().orc_switch_rows_k(_ptr(W_rows), _ptr(row_ids), n, out, inn, _ptr(A), _ptr(B),
+                                  r, float(s), k, _ptr(pi), _ptr(pg), _ptr(ci), _ptr(cg),
+                                  _ptr(W_new), _ptr(W_ex))
     if exact:
         return W_new, W_ex
     return W_new

@@ -31,14 +31,14 @@
  *   - merge scale s = alpha / r;
  *   - W_new = bf16_rne(W + dW), one rounding, with
  *     dW = s * sum_{e in cur} g_e B_e A_e  -  s * sum_{e in prev} g_e B_e A_e
- *     (each set has at most two terms, and a two-term fp64 sum does not
- *     depend on their order, so prev == cur cancels exactly).
+ *     (each set summed in slot order, so prev == cur cancels exactly).
  *
  * Layouts (row-major everywhere):
  *   h  [T, d] fp32, Wr [d, E] fp32
  *   W  [out, in] bf16 (as uint16 bit patterns)
  *   A  [E, r, in] bf16, B [E, out, r] bf16
- *   route: idx[2] int32 (-1 = no expert), gate[2] fp32
+ *   route: idx[k] int32 (-1 = no expert), gate[k] fp32; k = 2 for the
+ *   pages' top-2 router, 1..4 for the top-k widening
  */
 #include <math.h>
 #include <stdint.h>
@@ -128,15 +128,66 @@ void orc_pregate(const float* h, int64_t T, int64_t d, const float* Wr,
     }
 }
 
+/* Top-k pre-gating, k in [1, 4]: the same rule with k picks.  A reading of
+ * [P2] 2-ga beyond its top-2 router (the pages fix k = 2; larger k is the
+ * natural widening of the same router):
+ *   pick j = the largest z among the experts not yet picked, lowest index
+ *   among equals; p = softmax(z) over all E (max subtracted);
+ *   g_j = p_{e_j} / sum_{i < k} p_{e_i}, rounded to fp32.
+ * Slots past E hold idx -1 and gate 0.  idx_out / gate_out are [T, k]. */
+void orc_pregate_topk(const float* h, int64_t T, int64_t d, const float* Wr,
+                      int32_t E, int32_t k, int32_t* idx_out, float* gate_out,
+                      double* z_out) {
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        double* z = (double*)malloc(sizeof(double) * (size_t)E);
+        char* taken = (char*)calloc((size_t)E, 1);
+        for (int32_t e = 0; e < E; ++e) {
+            double acc = 0.0;
+            for (int64_t i = 0; i < d; ++i)
+                acc += (double)h[t * d + i] * (double)Wr[i * E + e];
+            z[e] = acc;
+        }
+        int32_t pick[4] = {-1, -1, -1, -1};
+        for (int32_t j = 0; j < k; ++j) {
+            int32_t best = -1;
+            for (int32_t e = 0; e < E; ++e) {
+                if (taken[e]) continue;
+                if (best < 0 || z[e] > z[best]) best = e;
+            }
+            if (best < 0) break;
+            pick[j] = best;
+            taken[best] = 1;
+        }
+        double zmax = z[pick[0]];
+        double denom = 0.0;
+        for (int32_t e = 0; e < E; ++e) denom += exp(z[e] - zmax);
+        double p[4] = {0.0, 0.0, 0.0, 0.0}, psum = 0.0;
+        for (int32_t j = 0; j < k; ++j)
+            if (pick[j] >= 0) {
+                p[j] = exp(z[pick[j]] - zmax) / denom;
+                psum += p[j];
+            }
+        for (int32_t j = 0; j < k; ++j) {
+            idx_out[t * k + j] = pick[j];
+            gate_out[t * k + j] = pick[j] >= 0 ? (float)(p[j] / psum) : 0.0f;
+        }
+        if (z_out)
+            for (int32_t e = 0; e < E; ++e) z_out[t * E + e] = z[e];
+        free(taken);
+        free(z);
+    }
+}
+
 /* ---- fused adapter switch ([P1] abstract, [P2] 2-na) -------------------- */
 
-/* The experts a route names (slots holding -1 are empty).  Returns how many
- * entries were written (0..2). */
-static int route_experts(const int32_t* idx, const float* gate, int32_t* e_out,
-                        double* g_out) {
+/* The experts a route of `slots` slots names (slots holding -1 are empty).
+ * Returns how many entries were written (0..slots). */
+static int route_experts(const int32_t* idx, const float* gate, int32_t slots,
+                        int32_t* e_out, double* g_out) {
     int n = 0;
     if (!idx) return 0;
-    for (int j = 0; j < 2; ++j) {
+    for (int j = 0; j < slots; ++j) {
         if (idx[j] < 0) continue;
         e_out[n] = idx[j];
         g_out[n] = (double)gate[j];
@@ -160,20 +211,25 @@ static double lora_product(const uint16_t* A, const uint16_t* B, int64_t out,
 /* One switch of one (layer, target) weight, on a chosen set of rows.
  *   W_rows   [n_rows, in]  the rows' values before the switch
  *   row_ids  [n_rows]      which rows of the [out, in] matrix they are
- *   prev_*, cur_*          a route (idx[2], gate[2]) or NULL for "none"
+ *   prev_*, cur_*          a route (idx[slots], gate[slots]) or NULL for "none"
+ *   slots                  route slots, 1..4 (the top-k of the router)
  *   W_new    [n_rows, in]  bf16_rne(W + dW)          (may be NULL)
  *   W_exact  [n_rows, in]  W + dW in fp64, unrounded (may be NULL)
- * dW = s * sum_{e in cur} g_e (B_e A_e) - s * sum_{e in prev} g_e (B_e A_e). */
-void orc_switch_rows(const uint16_t* W_rows, const int64_t* row_ids,
-                     int64_t n_rows, int64_t out, int64_t in,
-                     const uint16_t* A, const uint16_t* B, int32_t r, double s,
-                     const int32_t* prev_idx, const float* prev_gate,
-                     const int32_t* cur_idx, const float* cur_gate,
-                     uint16_t* W_new, double* W_exact) {
-    int32_t pe[2], ce[2];
-    double pg[2], cg[2];
-    int np = route_experts(prev_idx, prev_gate, pe, pg);
-    int nc = route_experts(cur_idx, cur_gate, ce, cg);
+ * dW = s * sum_{e in cur} g_e (B_e A_e) - s * sum_{e in prev} g_e (B_e A_e),
+ * each sum taken in slot order, so equal routes cancel exactly. */
+void orc_switch_rows_k(const uint16_t* W_rows, const int64_t* row_ids,
+                       int64_t n_rows, int64_t out, int64_t in,
+                       const uint16_t* A, const uint16_t* B, int32_t r, double s,
+                       int32_t slots,
+                       const int32_t* prev_idx, const float* prev_gate,
+                       const int32_t* cur_idx, const float* cur_gate,
+                       uint16_t* W_new, double* W_exact) {
+    int32_t pe[4], ce[4];
+    double pg[4], cg[4];
+    if (slots < 1) slots = 1;
+    if (slots > 4) slots = 4;
+    int np = route_experts(prev_idx, prev_gate, slots, pe, pg);
+    int nc = route_experts(cur_idx, cur_gate, slots, ce, cg);
 #pragma omp parallel for schedule(static)
     for (int64_t q = 0; q < n_rows; ++q) {
         int64_t i = row_ids[q];
@@ -189,6 +245,17 @@ void orc_switch_rows(const uint16_t* W_rows, const int64_t* row_ids,
             if (W_new) W_new[q * in + j] = orc_bf16_from_double(w);
         }
     }
+}
+
+/* The top-2 switch: routes of two slots. */
+void orc_switch_rows(const uint16_t* W_rows, const int64_t* row_ids,
+                     int64_t n_rows, int64_t out, int64_t in,
+                     const uint16_t* A, const uint16_t* B, int32_t r, double s,
+                     const int32_t* prev_idx, const float* prev_gate,
+                     const int32_t* cur_idx, const float* cur_gate,
+                     uint16_t* W_new, double* W_exact) {
+    orc_switch_rows_k(W_rows, row_ids, n_rows, out, in, A, B, r, s, 2, prev_idx,
+                      prev_gate, cur_idx, cur_gate, W_new, W_exact);
 }
 
 /* Threads the oracle's parallel loops use (1 when built without OpenMP). */
