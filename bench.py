@@ -51,6 +51,9 @@ def parse():
                          "mma.sync (mma), or auto")
     ap.add_argument("--mode", choices=["switch", "rebase"], default="switch",
                     help="in-place switch (prev -> cur) or re-base from a pristine copy W0")
+    ap.add_argument("--top-k", type=int, default=2,
+                    help="experts per token: 2 is the top-2 router and route record; 1..4 "
+                         "uses the top-k entry points (an in-place switch touches up to 2k)")
     ap.add_argument("--router-tokens", type=int, default=4096,
                     help="also time the pre-gate alone on this many tokens (0 = skip)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -265,11 +268,11 @@ def oracle_rate(cfg, target_s=10.0, seed_layers=1):
     return gbs, oracle.num_threads(), desc, dt, elems
 
 
-def workload_label(cfg, n_tokens):
+def workload_label(cfg, n_tokens, top_k=2):
     from weight_merge_b200 import workloads as wl
     return (f"{cfg.name}: {cfg.shape}, {cfg.n_layers} layers x {len(cfg.targets)} targets "
             f"({wl.describe_targets(cfg)}), E={cfg.n_experts}, r={cfg.rank}, "
-            f"alpha={cfg.alpha:g}, top-2, {n_tokens}-token decode switch sequence")
+            f"alpha={cfg.alpha:g}, top-{top_k}, {n_tokens}-token decode switch sequence")
 
 
 # --------------------------------------------------------------------------
@@ -360,7 +363,15 @@ def run_ours(args):
         sw.set_base([w.clone() for w in model.W])
     T = cfg.n_tokens
     h = wl.make_hidden(cfg, T=T, device="cuda")
-    routes = torch.zeros((T, 4), dtype=torch.int32, device="cuda")
+    topk = args.top_k != 2
+    routes = torch.zeros((T, 8 if topk else 4), dtype=torch.int32, device="cuda")
+    rptr = B.Switcher.route4_ptr if topk else B.Switcher.route_ptr
+
+    def pregate(hh, r_rows):
+        if topk:
+            sw.pregate_topk(hh, model.Wr, args.top_k, r_rows, sh)
+        else:
+            sw.pregate(hh, model.Wr, r_rows, sh)
     stream = torch.cuda.current_stream()
     sh = stream.cuda_stream
     w_bytes = cfg.w_bytes_per_switch()
@@ -371,13 +382,13 @@ def run_ours(args):
 
     def do_switch(prev_t, t):
         if rebase:
-            sw.rebase(B.Switcher.route_ptr(routes, t), sh)
+            (sw.rebase_topk if topk else sw.rebase)(rptr(routes, t), sh)
         else:
-            sw.switch(B.Switcher.route_ptr(routes, prev_t), B.Switcher.route_ptr(routes, t), sh)
+            (sw.switch_topk if topk else sw.switch)(rptr(routes, prev_t), rptr(routes, t), sh)
 
     def step(k, prev_t):
         t = k % T
-        sw.pregate(h[t:t + 1], model.Wr, routes[t:t + 1], sh)
+        pregate(h[t:t + 1], routes[t:t + 1])
         do_switch(prev_t, t)
         return t
 
@@ -404,7 +415,7 @@ def run_ours(args):
             kk = args.warmup + k
             t = kk % T
             st_start[k].record(stream)
-            sw.pregate(h[t:t + 1], model.Wr, routes[t:t + 1], sh)
+            pregate(h[t:t + 1], routes[t:t + 1])
             sw_start[k].record(stream)
             do_switch(prev_t, t)
             sw_end[k].record(stream)
@@ -437,7 +448,7 @@ def run_ours(args):
     e2e = None
     if not args.no_e2e:
         h_host = h.cpu().pin_memory()
-        r_host = torch.zeros((1, 4), dtype=torch.int32).pin_memory()
+        r_host = torch.zeros((1, routes.shape[1]), dtype=torch.int32).pin_memory()
         h_dev = torch.empty((1, cfg.d), dtype=torch.float32, device="cuda")
         ev0 = torch.cuda.Event(enable_timing=True)
         ev1 = torch.cuda.Event(enable_timing=True)
@@ -448,7 +459,7 @@ def run_ours(args):
         for k in range(args.steps):
             t = (args.warmup + args.steps + k) % T
             h_dev.copy_(h_host[t:t + 1], non_blocking=True)
-            sw.pregate(h_dev, model.Wr, routes[t:t + 1], sh)
+            pregate(h_dev, routes[t:t + 1])
             do_switch(pe, t)
             r_host.copy_(routes[t:t + 1], non_blocking=True)
             pe = t
@@ -465,7 +476,8 @@ def run_ours(args):
             pp = t
         e_max, e_units = reduce_over_ranks(e_ms, e_real, world, device="cuda")
         e2e = {"value": round(e_units * w_bytes / (e_max / 1000) / 1e9, 2),
-               "unit": "GB/s", "h2d_bytes_per_step": cfg.d * 4, "d2h_bytes_per_step": 16}
+               "unit": "GB/s", "h2d_bytes_per_step": cfg.d * 4,
+               "d2h_bytes_per_step": 4 * routes.shape[1]}
 
     # the router alone on a batch of tokens (the Llama-3-8B-shaped router
     # batch: T=4096, d=4096, E=8): an HBM-bound GEMV over h
@@ -516,7 +528,7 @@ def run_ours(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded random weights and hidden states)",
             "config": {
-                "workload": workload_label(cfg, T),
+                "workload": workload_label(cfg, T, args.top_k),
                 "w_bytes_per_switch": w_bytes,
                 "l2": "inputs larger than L2 (W read+write per switch >> 126 MB), no flush",
                 "parallelism": f"replicas x{world}",

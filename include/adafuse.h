@@ -97,6 +97,18 @@ typedef struct adafuse_route {
     float gate[2];
 } adafuse_route;
 
+/* A top-k routing decision, k in [1, ADAFUSE_MAX_TOP_K] (32 bytes): the k
+ * chosen experts in order and their gates; slots past k, or past the number
+ * of experts, hold idx -1 (their gate is ignored).  adafuse_pregate_topk
+ * writes non-increasing gates that sum to 1 up to rounding.  The pages'
+ * router is top-2 (gist.science technical summary, section 2-ga); top-k is
+ * the same router widened to k picks. */
+#define ADAFUSE_MAX_TOP_K 4
+typedef struct adafuse_route4 {
+    int32_t idx[4];
+    float gate[4];
+} adafuse_route4;
+
 /* One LoRA-targeted weight of one layer (for example q_proj of layer 7).
  *   out, in  W's shape; both multiples of 8.
  *   W        device pointer, [out, in] bf16, 16-byte aligned, updated in place.
@@ -210,6 +222,37 @@ ADAFUSE_API int adafuse_rebase(adafuse_ctx* ctx, const adafuse_route* cur, void*
 /* As adafuse_rebase, restricted to layers [layer_begin, layer_begin + n_layers). */
 ADAFUSE_API int adafuse_rebase_layers(adafuse_ctx* ctx, int32_t layer_begin, int32_t n_layers,
                                       const adafuse_route* cur, void* stream);
+
+/* ---- top-k routing --------------------------------------------------------
+ * The router and the switches above with k in [1, 4] experts per token.  An
+ * in-place switch then touches up to 2k experts (k leaving, k arriving). */
+
+/* Top-k pre-gating: as adafuse_pregate, with route[t] the k experts first
+ * under (logit descending, index ascending) and gates g_j = the softmax over
+ * all experts renormalised over the k picks.  k outside [1, 4] is
+ * INVALID_ARG.  route: device array of T adafuse_route4, 16-byte aligned.
+ * For k = 2 the experts and gates equal adafuse_pregate's bit for bit.  A
+ * token's route does not depend on the batch it is gated in. */
+ADAFUSE_API int adafuse_pregate_topk(adafuse_ctx* ctx, const float* h, int64_t T, int64_t d,
+                                     const float* Wr, int32_t k, adafuse_route4* route,
+                                     void* stream);
+
+/* As adafuse_switch with top-k routes: per expert e in prev U cur the
+ * coefficient is c_e = s*(g_cur(e) - g_prev(e)), experts with c_e == 0 are
+ * dropped, and W <- bf16_rne(W + sum_e c_e B_e A_e) with fp32 accumulation
+ * (up to 8 experts in one launch).  prev / cur: 16-byte aligned device
+ * routes or NULL.  Bad routes set the status word and write nothing. */
+ADAFUSE_API int adafuse_switch_topk(adafuse_ctx* ctx, const adafuse_route4* prev,
+                                    const adafuse_route4* cur, void* stream);
+
+/* As adafuse_switch_topk, restricted to layers [layer_begin, layer_begin + n_layers). */
+ADAFUSE_API int adafuse_switch_topk_layers(adafuse_ctx* ctx, int32_t layer_begin,
+                                           int32_t n_layers, const adafuse_route4* prev,
+                                           const adafuse_route4* cur, void* stream);
+
+/* As adafuse_rebase with a top-k route: W <- bf16_rne(W0 + s*sum_{e in cur}
+ * g_e B_e A_e).  INVALID_ARG without a registered base. */
+ADAFUSE_API int adafuse_rebase_topk(adafuse_ctx* ctx, const adafuse_route4* cur, void* stream);
 
 /* Synchronise `stream`, read the device status word into *status, then
  * clear it.  Returns ADAFUSE_ERR_DEVICE_FAULT when the word was non-zero,

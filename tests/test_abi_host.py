@@ -108,6 +108,10 @@ def test_calls_on_null_context_are_invalid():
     assert L.adafuse_pregate(None, None, 1, 8, None, None, None) == B.ADAFUSE_ERR_INVALID_ARG
     st = ctypes.c_int32()
     assert L.adafuse_get_device_status(None, None, ctypes.byref(st)) == B.ADAFUSE_ERR_INVALID_ARG
+    assert L.adafuse_pregate_topk(None, None, 1, 8, None, 2, None, None) == B.ADAFUSE_ERR_INVALID_ARG
+    assert L.adafuse_switch_topk(None, None, None, None) == B.ADAFUSE_ERR_INVALID_ARG
+    assert L.adafuse_switch_topk_layers(None, 0, 1, None, None, None) == B.ADAFUSE_ERR_INVALID_ARG
+    assert L.adafuse_rebase_topk(None, None, None) == B.ADAFUSE_ERR_INVALID_ARG
     assert L.adafuse_destroy(None) == B.ADAFUSE_OK
 
 

@@ -28,6 +28,7 @@ ADAFUSE_KERNEL_AUTO = 0
 ADAFUSE_KERNEL_MMA_SYNC = 1
 ADAFUSE_KERNEL_TCGEN05 = 2
 ADAFUSE_KERNEL_TCGEN05_PAIR = 3
+ADAFUSE_MAX_TOP_K = 4
 
 
 class AdafuseError(RuntimeError):
@@ -41,6 +42,10 @@ class AdafuseError(RuntimeError):
 
 class Route(ctypes.Structure):
     _fields_ = [("idx", ctypes.c_int32 * 2), ("gate", ctypes.c_float * 2)]
+
+
+class Route4(ctypes.Structure):
+    _fields_ = [("idx", ctypes.c_int32 * 4), ("gate", ctypes.c_float * 4)]
 
 
 class Target(ctypes.Structure):
@@ -85,6 +90,10 @@ def lib() -> ctypes.CDLL:
         "adafuse_rebase": ([P, P, P], ctypes.c_int),
         "adafuse_rebase_layers": ([P, i32, i32, P, P], ctypes.c_int),
         "adafuse_get_switch_kernel": ([P], ctypes.c_int),
+        "adafuse_pregate_topk": ([P, P, i64, i64, P, i32, P, P], ctypes.c_int),
+        "adafuse_switch_topk": ([P, P, P, P], ctypes.c_int),
+        "adafuse_switch_topk_layers": ([P, i32, i32, P, P, P], ctypes.c_int),
+        "adafuse_rebase_topk": ([P, P, P], ctypes.c_int),
         "adafuse_segment_table": ([ctypes.POINTER(Desc), P, i64, ctypes.POINTER(i64)], ctypes.c_int),
         "adafuse_tile_size": ([], ctypes.c_int),
         "adafuse_strerror": ([ctypes.c_int], ctypes.c_char_p),
@@ -157,6 +166,28 @@ def adafuse_rebase_layers(ctx: int, layer_begin: int, n_layers: int, cur: Option
                           stream: int = 0) -> None:
     _check(lib().adafuse_rebase_layers(ctx, int(layer_begin), int(n_layers), cur or None,
                                        stream or None), "adafuse_rebase_layers")
+
+
+def adafuse_pregate_topk(ctx: int, h: int, T: int, d: int, Wr: int, k: int, route: int,
+                         stream: int = 0) -> None:
+    _check(lib().adafuse_pregate_topk(ctx, h, int(T), int(d), Wr, int(k), route, stream or None),
+           "adafuse_pregate_topk")
+
+
+def adafuse_switch_topk(ctx: int, prev: Optional[int], cur: Optional[int], stream: int = 0) -> None:
+    _check(lib().adafuse_switch_topk(ctx, prev or None, cur or None, stream or None),
+           "adafuse_switch_topk")
+
+
+def adafuse_switch_topk_layers(ctx: int, layer_begin: int, n_layers: int, prev: Optional[int],
+                               cur: Optional[int], stream: int = 0) -> None:
+    _check(lib().adafuse_switch_topk_layers(ctx, int(layer_begin), int(n_layers), prev or None,
+                                            cur or None, stream or None),
+           "adafuse_switch_topk_layers")
+
+
+def adafuse_rebase_topk(ctx: int, cur: Optional[int], stream: int = 0) -> None:
+    _check(lib().adafuse_rebase_topk(ctx, cur or None, stream or None), "adafuse_rebase_topk")
 
 
 def adafuse_set_switch_kernel(ctx: int, kernel: int) -> None:
@@ -258,6 +289,28 @@ class Switcher:
     def rebase_layers(self, layer_begin: int, n_layers: int, cur: Optional[int],
                       stream: int = 0) -> None:
         adafuse_rebase_layers(self.ctx, layer_begin, n_layers, cur, stream)
+
+    @staticmethod
+    def route4_ptr(routes, t: Optional[int]) -> Optional[int]:
+        """Device address of route t of a [T, 8] int32 top-k route buffer."""
+        if t is None or routes is None:
+            return None
+        return routes.data_ptr() + 32 * int(t)
+
+    def pregate_topk(self, h, Wr, k: int, routes, stream: int = 0) -> None:
+        T, d = h.shape
+        adafuse_pregate_topk(self.ctx, h.data_ptr(), T, d, Wr.data_ptr(), k, routes.data_ptr(),
+                             stream)
+
+    def switch_topk(self, prev: Optional[int], cur: Optional[int], stream: int = 0) -> None:
+        adafuse_switch_topk(self.ctx, prev, cur, stream)
+
+    def switch_topk_layers(self, layer_begin: int, n_layers: int, prev: Optional[int],
+                           cur: Optional[int], stream: int = 0) -> None:
+        adafuse_switch_topk_layers(self.ctx, layer_begin, n_layers, prev, cur, stream)
+
+    def rebase_topk(self, cur: Optional[int], stream: int = 0) -> None:
+        adafuse_rebase_topk(self.ctx, cur, stream)
 
     def set_kernel(self, kernel: int) -> None:
         adafuse_set_switch_kernel(self.ctx, kernel)

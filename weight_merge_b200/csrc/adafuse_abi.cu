@@ -131,8 +131,8 @@ bool pair_eligible(const adafuse_ctx* c) { return c->tc_kp != 0 && c->rank != 8;
 int kp_class(int r) { return r <= 8 ? 8 : r <= 16 ? 16 : r <= 32 ? 32 : 64; }
 
 template <int KP, bool BBULK>
-cudaError_t launch_tc(const adafuse_ctx* c, int64_t t0, int64_t t1, const adafuse_route* prev,
-                      const adafuse_route* cur, cudaStream_t s, bool rebase) {
+cudaError_t launch_tc(const adafuse_ctx* c, int64_t t0, int64_t t1, const int32_t* prev,
+                      const int32_t* cur, int slots, cudaStream_t s, bool rebase) {
     TcParams prm;
     prm.pairs = c->d_pairs;
     prm.tiles = c->d_tiles;
@@ -141,6 +141,7 @@ cudaError_t launch_tc(const adafuse_ctx* c, int64_t t0, int64_t t1, const adafus
     prm.t_end = t1;
     prm.prev = prev;
     prm.cur = cur;
+    prm.slots = slots;
     prm.E = c->n_experts;
     prm.s = c->scale;
     prm.status = c->d_status;
@@ -150,8 +151,8 @@ cudaError_t launch_tc(const adafuse_ctx* c, int64_t t0, int64_t t1, const adafus
 }
 
 template <int KP>
-cudaError_t launch_tc2(adafuse_ctx* c, int64_t b0, int64_t b1, const adafuse_route* prev,
-                       const adafuse_route* cur, cudaStream_t s, bool rebase) {
+cudaError_t launch_tc2(adafuse_ctx* c, int64_t b0, int64_t b1, const int32_t* prev,
+                       const int32_t* cur, int slots, cudaStream_t s, bool rebase) {
     if (c->pair_clusters == 0) {
         const cudaError_t e = pair_kernel_clusters<KP>(c->sm_count, &c->pair_clusters);
         if (e != cudaSuccess) {
@@ -167,6 +168,7 @@ cudaError_t launch_tc2(adafuse_ctx* c, int64_t b0, int64_t b1, const adafuse_rou
     prm.t_end = b1;
     prm.prev = prev;
     prm.cur = cur;
+    prm.slots = slots;
     prm.E = c->n_experts;
     prm.s = c->scale;
     prm.status = c->d_status;
@@ -394,8 +396,15 @@ int adafuse_get_switch_kernel(adafuse_ctx* ctx) {
     return ctx->kernel;
 }
 
-int adafuse_pregate(adafuse_ctx* ctx, const float* h, int64_t T, int64_t d, const float* Wr,
-                    adafuse_route* route, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Top-k pre-gating into routes of `slots` slots (2: adafuse_route, 4:
+// adafuse_route4).  The same kernels and arithmetic for every k and batch.
+int pregate_launch(adafuse_ctx* ctx, const float* h, int64_t T, int64_t d, const float* Wr,
+                   int k, int slots, void* route_out, void* stream) {
+    int32_t* route = static_cast<int32_t*>(route_out);
     if (ctx == nullptr || T < 0 || d < 1 || (d & 3) != 0) return ADAFUSE_ERR_INVALID_ARG;
     if (T == 0) return ADAFUSE_OK;
     if (h == nullptr || Wr == nullptr || route == nullptr) return ADAFUSE_ERR_INVALID_ARG;
@@ -415,7 +424,7 @@ int adafuse_pregate(adafuse_ctx* ctx, const float* h, int64_t T, int64_t d, cons
     const unsigned grid = (unsigned)(shared ? std::min<int64_t>(groups, (int64_t)ctx->sm_count) : groups);
     auto go = [&](auto kernel, size_t smem) {
         if (smem > 0) cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        kernel<<<grid, kPregateThreads, smem, s>>>(h, T, d, Wr, E, route);
+        kernel<<<grid, kPregateThreads, smem, s>>>(h, T, d, Wr, E, k, slots, route);
     };
     if (shared) {
         switch (emax) {
@@ -443,6 +452,21 @@ int adafuse_pregate(adafuse_ctx* ctx, const float* h, int64_t T, int64_t d, cons
     return e == cudaSuccess ? ADAFUSE_OK : cuda_fail(e, "pregate launch");
 }
 
+}  // namespace
+
+extern "C" {
+
+int adafuse_pregate(adafuse_ctx* ctx, const float* h, int64_t T, int64_t d, const float* Wr,
+                    adafuse_route* route, void* stream) {
+    return pregate_launch(ctx, h, T, d, Wr, 2, 2, route, stream);
+}
+
+int adafuse_pregate_topk(adafuse_ctx* ctx, const float* h, int64_t T, int64_t d,
+                         const float* Wr, int32_t k, adafuse_route4* route, void* stream) {
+    if (k < 1 || k > ADAFUSE_MAX_TOP_K) return ADAFUSE_ERR_INVALID_ARG;
+    return pregate_launch(ctx, h, T, d, Wr, k, 4, route, stream);
+}
+
 }  // extern "C"
 
 namespace {
@@ -450,7 +474,10 @@ namespace {
 // One switch launch over layers [layer_begin, layer_begin + n_layers): in
 // place (prev, cur) or, with rebase, W <- rne(W0 + dW_cur).
 int launch_switch(adafuse_ctx* ctx, int32_t layer_begin, int32_t n_layers,
-                  const adafuse_route* prev, const adafuse_route* cur, void* stream, bool rebase) {
+                  const void* prev_route, const void* cur_route, int slots, void* stream,
+                  bool rebase) {
+    const int32_t* prev = static_cast<const int32_t*>(prev_route);
+    const int32_t* cur = static_cast<const int32_t*>(cur_route);
     if (ctx == nullptr || n_layers < 0 || layer_begin < 0) return ADAFUSE_ERR_INVALID_ARG;
     if ((int64_t)layer_begin + n_layers > ctx->n_layers) return ADAFUSE_ERR_INVALID_ARG;
     if (!aligned16(prev) || !aligned16(cur)) return ADAFUSE_ERR_INVALID_ARG;
@@ -467,23 +494,23 @@ int launch_switch(adafuse_ctx* ctx, int32_t layer_begin, int32_t n_layers,
         const int64_t b1 = ctx->layer_block_begin[(size_t)layer_begin + n_layers];
         cudaError_t e = cudaSuccess;
         if (ctx->tc_kp == 16)
-            e = launch_tc2<16>(ctx, b0, b1, prev, cur, s, rebase);
+            e = launch_tc2<16>(ctx, b0, b1, prev, cur, slots, s, rebase);
         else if (ctx->tc_kp == 32)
-            e = launch_tc2<32>(ctx, b0, b1, prev, cur, s, rebase);
+            e = launch_tc2<32>(ctx, b0, b1, prev, cur, slots, s, rebase);
         else
-            e = launch_tc2<64>(ctx, b0, b1, prev, cur, s, rebase);
+            e = launch_tc2<64>(ctx, b0, b1, prev, cur, slots, s, rebase);
         return e == cudaSuccess ? ADAFUSE_OK : cuda_fail(e, "switch launch");
     }
     if (kind == ADAFUSE_KERNEL_TCGEN05) {
         cudaError_t e = cudaSuccess;
         if (ctx->rank == 8)
-            e = launch_tc<16, true>(ctx, t0, t1, prev, cur, s, rebase);
+            e = launch_tc<16, true>(ctx, t0, t1, prev, cur, slots, s, rebase);
         else if (ctx->tc_kp == 16)
-            e = launch_tc<16, false>(ctx, t0, t1, prev, cur, s, rebase);
+            e = launch_tc<16, false>(ctx, t0, t1, prev, cur, slots, s, rebase);
         else if (ctx->tc_kp == 32)
-            e = launch_tc<32, false>(ctx, t0, t1, prev, cur, s, rebase);
+            e = launch_tc<32, false>(ctx, t0, t1, prev, cur, slots, s, rebase);
         else
-            e = launch_tc<64, false>(ctx, t0, t1, prev, cur, s, rebase);
+            e = launch_tc<64, false>(ctx, t0, t1, prev, cur, slots, s, rebase);
         return e == cudaSuccess ? ADAFUSE_OK : cuda_fail(e, "switch launch");
     }
     const int64_t want = (int64_t)ctx->sm_count * 2;
@@ -491,23 +518,16 @@ int launch_switch(adafuse_ctx* ctx, int32_t layer_begin, int32_t n_layers,
     const int E = ctx->n_experts, r = ctx->rank;
     const float sc = ctx->scale;
     const int rb = rebase ? 1 : 0;
+    auto go = [&](auto kernel) {
+        kernel<<<grid, kSwitchThreads, 0, s>>>(ctx->d_pairs, ctx->d_tiles, t0, t1, prev, cur, E, r,
+                                               sc, ctx->d_status, rb);
+    };
+    const bool four = slots == 4;
     switch (kp_class(r)) {
-        case 8:
-            switch_mma_kernel<8><<<grid, kSwitchThreads, 0, s>>>(ctx->d_pairs, ctx->d_tiles, t0, t1,
-                                                                 prev, cur, E, r, sc, ctx->d_status, rb);
-            break;
-        case 16:
-            switch_mma_kernel<16><<<grid, kSwitchThreads, 0, s>>>(ctx->d_pairs, ctx->d_tiles, t0, t1,
-                                                                  prev, cur, E, r, sc, ctx->d_status, rb);
-            break;
-        case 32:
-            switch_mma_kernel<32><<<grid, kSwitchThreads, 0, s>>>(ctx->d_pairs, ctx->d_tiles, t0, t1,
-                                                                  prev, cur, E, r, sc, ctx->d_status, rb);
-            break;
-        default:
-            switch_mma_kernel<64><<<grid, kSwitchThreads, 0, s>>>(ctx->d_pairs, ctx->d_tiles, t0, t1,
-                                                                  prev, cur, E, r, sc, ctx->d_status, rb);
-            break;
+        case 8: four ? go(switch_mma_kernel<8, 4>) : go(switch_mma_kernel<8, 2>); break;
+        case 16: four ? go(switch_mma_kernel<16, 4>) : go(switch_mma_kernel<16, 2>); break;
+        case 32: four ? go(switch_mma_kernel<32, 4>) : go(switch_mma_kernel<32, 2>); break;
+        default: four ? go(switch_mma_kernel<64, 4>) : go(switch_mma_kernel<64, 2>); break;
     }
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? ADAFUSE_OK : cuda_fail(e, "switch launch");
@@ -520,7 +540,7 @@ extern "C" {
 int adafuse_switch_batch_layers(adafuse_ctx* ctx, int32_t layer_begin, int32_t n_layers,
                                 const adafuse_route* prev, const adafuse_route* cur,
                                 void* stream) {
-    return launch_switch(ctx, layer_begin, n_layers, prev, cur, stream, false);
+    return launch_switch(ctx, layer_begin, n_layers, prev, cur, 2, stream, false);
 }
 
 int adafuse_set_base(adafuse_ctx* ctx, const void* const* W0) {
@@ -575,7 +595,7 @@ int adafuse_set_base(adafuse_ctx* ctx, const void* const* W0) {
 int adafuse_rebase_layers(adafuse_ctx* ctx, int32_t layer_begin, int32_t n_layers,
                           const adafuse_route* cur, void* stream) {
     if (ctx == nullptr || !ctx->has_base) return ADAFUSE_ERR_INVALID_ARG;
-    return launch_switch(ctx, layer_begin, n_layers, nullptr, cur, stream, true);
+    return launch_switch(ctx, layer_begin, n_layers, nullptr, cur, 2, stream, true);
 }
 
 int adafuse_rebase(adafuse_ctx* ctx, const adafuse_route* cur, void* stream) {
@@ -587,6 +607,23 @@ int adafuse_switch(adafuse_ctx* ctx, const adafuse_route* prev, const adafuse_ro
                    void* stream) {
     if (ctx == nullptr) return ADAFUSE_ERR_INVALID_ARG;
     return adafuse_switch_batch_layers(ctx, 0, ctx->n_layers, prev, cur, stream);
+}
+
+int adafuse_switch_topk_layers(adafuse_ctx* ctx, int32_t layer_begin, int32_t n_layers,
+                               const adafuse_route4* prev, const adafuse_route4* cur,
+                               void* stream) {
+    return launch_switch(ctx, layer_begin, n_layers, prev, cur, 4, stream, false);
+}
+
+int adafuse_switch_topk(adafuse_ctx* ctx, const adafuse_route4* prev, const adafuse_route4* cur,
+                        void* stream) {
+    if (ctx == nullptr) return ADAFUSE_ERR_INVALID_ARG;
+    return adafuse_switch_topk_layers(ctx, 0, ctx->n_layers, prev, cur, stream);
+}
+
+int adafuse_rebase_topk(adafuse_ctx* ctx, const adafuse_route4* cur, void* stream) {
+    if (ctx == nullptr || !ctx->has_base) return ADAFUSE_ERR_INVALID_ARG;
+    return launch_switch(ctx, 0, ctx->n_layers, nullptr, cur, 4, stream, true);
 }
 
 int adafuse_get_device_status(adafuse_ctx* ctx, void* stream, int32_t* status) {

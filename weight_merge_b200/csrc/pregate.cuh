@@ -32,7 +32,7 @@ enum : int { kWrShared = 0, kWrVector = 1, kWrScalar = 2 };
 template <int EMAX, int TPB, int WR>
 __global__ void __launch_bounds__(kPregateThreads)
 pregate_kernel(const float* __restrict__ h, int64_t T, int64_t d, const float* __restrict__ Wr,
-               int E, adafuse_route* __restrict__ route) {
+               int E, int k, int slots, int32_t* __restrict__ route) {
     static_assert(EMAX % 4 == 0, "EMAX");
     constexpr int kWarps = kPregateThreads / 32;
     constexpr int S4 = EMAX + 1;             // float4 slots per chunk in shared memory
@@ -127,30 +127,48 @@ pregate_kernel(const float* __restrict__ h, int64_t T, int64_t d, const float* _
                 for (int w = 1; w < kWarps; ++w) v += part[w][tt][e];
                 z[e] = v;
             }
-            // top-2 under (z descending, index ascending)
-            int e0 = 0;
-            float z0 = z[0];
+            // top-k under (z descending, index ascending): pick j is the
+            // largest logit not yet picked, the lower index among equals
+            int pick[4] = {-1, -1, -1, -1};
+            float zp[4] = {0.f, 0.f, 0.f, 0.f};
+            uint64_t taken = 0;
 #pragma unroll
-            for (int e = 1; e < EMAX; ++e)
-                if (e < E && z[e] > z0) { e0 = e; z0 = z[e]; }
-            int e1 = -1;
-            float z1 = 0.f;
+            for (int j = 0; j < 4; ++j) {
+                if (j >= k) break;
+                int best = -1;
+                float zb = 0.f;
 #pragma unroll
-            for (int e = 0; e < EMAX; ++e) {
-                if (e >= E || e == e0) continue;
-                if (e1 < 0 || z[e] > z1) { e1 = e; z1 = z[e]; }
+                for (int e = 0; e < EMAX; ++e) {
+                    if (e >= E || ((taken >> e) & 1ull)) continue;
+                    if (best < 0 || z[e] > zb) { best = e; zb = z[e]; }
+                }
+                if (best < 0) break;
+                pick[j] = best;
+                zp[j] = zb;
+                taken |= 1ull << best;
             }
-            float g0 = 1.f, g1 = 0.f;
-            if (e1 >= 0) {
-                // softmax over all E renormalised over the picks == softmax of
-                // the two logits: g0 = 1 / (1 + exp(z1 - z0)), z1 - z0 <= 0.
-                const float x = expf(z1 - z0);
-                const float den = 1.f + x;
-                g0 = 1.f / den;
-                g1 = x / den;
+            // softmax over all E renormalised over the picks == softmax of the
+            // picked logits: g_j = x_j / (1 + x_1 + ...), x_j = exp(z_j - z_0) <= 1
+            float x[4] = {1.f, 0.f, 0.f, 0.f};
+            float den = 1.f;
+#pragma unroll
+            for (int j = 1; j < 4; ++j)
+                if (pick[j] >= 0) {
+                    x[j] = expf(zp[j] - zp[0]);
+                    den = den + x[j];
+                }
+            float g[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) g[j] = pick[j] >= 0 ? x[j] / den : 0.f;
+            if (slots == 2) {
+                reinterpret_cast<int4*>(route)[t0 + tt] =
+                    make_int4(pick[0], pick[1], __float_as_int(g[0]), __float_as_int(g[1]));
+            } else {
+                int4* r4 = reinterpret_cast<int4*>(route) + 2 * (t0 + tt);
+                r4[0] = make_int4(pick[0], pick[1], pick[2], pick[3]);
+                r4[1] = make_int4(__float_as_int(g[0]), __float_as_int(g[1]), __float_as_int(g[2]),
+                                  __float_as_int(g[3]));
             }
-            reinterpret_cast<int4*>(route)[t0 + tt] =
-                make_int4(e0, e1, __float_as_int(g0), __float_as_int(g1));
         }
         __syncthreads();   // part[] is reused by the next token group
     }

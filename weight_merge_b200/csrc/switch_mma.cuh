@@ -112,13 +112,14 @@ __device__ __forceinline__ TileCoord load_tile(const PairDesc* __restrict__ pair
 // KP: per-expert contraction depth rounded up to 8, 16, 32 or 64.
 // rebase: read W from the pristine base W0 instead of W itself (prev is null),
 // so W <- rne(W0 + dW_cur); then even an empty route writes (it copies W0).
-template <int KP>
+// SLOTS: route slots (2 for top-2 routes, 4 for top-k), so at most 2 * SLOTS experts.
+template <int KP, int SLOTS>
 __global__ void __launch_bounds__(kSwitchThreads, 2)
 switch_mma_kernel(const PairDesc* __restrict__ pairs, const TileEntry* __restrict__ tiles,
-                  int64_t t_begin, int64_t t_end, const adafuse_route* prev,
-                  const adafuse_route* cur, int E, int r, float s, int32_t* status, int rebase) {
-    Coefs cf;
-    const int st = build_coefs(prev, cur, E, s, cf);
+                  int64_t t_begin, int64_t t_end, const int32_t* prev, const int32_t* cur,
+                  int E, int r, float s, int32_t* status, int rebase) {
+    CoefsT<2 * SLOTS> cf;
+    const int st = build_coefs_slots<SLOTS>(prev, cur, E, s, cf);
     if (st != 0) {
         if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(status, st);
         return;
@@ -166,7 +167,7 @@ switch_mma_kernel(const PairDesc* __restrict__ pairs, const TileEntry* __restric
                 for (int q = 0; q < 4; ++q) tot[j][q] = 0.f;
 
 #pragma unroll
-            for (int ei = 0; ei < 4; ++ei) {
+            for (int ei = 0; ei < 2 * SLOTS; ++ei) {
                 if (ei >= cf.n) break;
                 const int e = cf.e[ei];
                 const uint16_t* Be = tc.B + (int64_t)e * tc.out * r;

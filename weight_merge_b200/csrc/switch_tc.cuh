@@ -80,8 +80,9 @@ struct TcParams {
     const TileEntry* tiles;
     const CUtensorMap* maps;  // 3 per pair: W, A, B
     int64_t t_begin, t_end;
-    const adafuse_route* prev;
-    const adafuse_route* cur;
+    const int32_t* prev;  // routes of `slots` slots (adafuse_route or adafuse_route4)
+    const int32_t* cur;
+    int slots;
     int E;
     float s;
     int32_t* status;
@@ -114,15 +115,23 @@ __device__ __forceinline__ TileInfo decode_tile(TileEntry te) {
 }
 
 // Epilogue arithmetic shared by both tensor-core kernels, for one thread's row
-// and 32-column group.
-//   tot = sum_e c_e * acc_e   (experts in order, fused multiply-add in fp32)
-__device__ __forceinline__ void epi_combine(uint32_t t_lane, const Coefs& cf, float (&tot)[32]) {
+// and 32-column group.  TMEM holds at most four 128-column accumulators, so
+// the experts of a switch come in batches of up to four (kTmemBatch):
+//   tot += sum_{e in batch} c_e * acc_e   (experts in order, fp32 FMA)
+constexpr int kTmemBatch = 4;
+
+// Batches per tile: at least one, so that a re-base with an empty route still
+// passes every tile through the epilogue.
+__device__ __forceinline__ int tmem_batches(const Coefs8& cf) {
+    return cf.n == 0 ? 1 : (cf.n + kTmemBatch - 1) / kTmemBatch;
+}
+
+__device__ __forceinline__ void epi_combine(uint32_t t_lane, const Coefs8& cf, int b0,
+                                            float (&tot)[32]) {
 #pragma unroll
-    for (int i = 0; i < 32; ++i) tot[i] = 0.f;
-#pragma unroll
-    for (int ei = 0; ei < 4; ++ei) {
-        if (ei < cf.n) {
-            const float c = cf.c[ei];
+    for (int ei = 0; ei < kTmemBatch; ++ei) {
+        if (b0 + ei < cf.n) {
+            const float c = coef_value(cf, b0 + ei);
             float v[32];
             sm100::tmem_ld32(t_lane + 128u * ei, v);
             sm100::tmem_wait_ld();
@@ -177,8 +186,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epi_done + C::kWStages);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-    Coefs cf;
-    const int st = build_coefs(p.prev, p.cur, p.E, p.s, cf);
+    Coefs8 cf;
+    const int st = build_coefs(p.prev, p.cur, p.slots, p.E, p.s, cf);
     if (st != 0) {
         if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(p.status, st);
         return;
@@ -288,7 +297,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
                 bool ok = true;
 #pragma unroll 1
                 for (int ei = 0; ei < cf.n; ++ei) {
-                    const int e = ei == 0 ? cf.e[0] : ei == 1 ? cf.e[1] : ei == 2 ? cf.e[2] : cf.e[3];
+                    const int e = coef_expert(cf, ei);
                     if (!mbar_wait_bounded(&op_empty[os], oph ^ 1, abort_flag, kWaitLimitNs)) { ok = false; break; }
                     uint8_t* a_dst = op_ring + (size_t)os * C::kOpStageBytes;
                     uint8_t* b_dst = a_dst + C::kABytes;
@@ -321,12 +330,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
             const uint32_t zero_s = smem_u32(zero_blk);
             int os = 0;
             uint32_t oph = 0, aph = 0;
-            for (int64_t t = first; t < p.t_end && !*abort_flag; t += gridDim.x) {
-                if (!mbar_wait_bounded(acc_empty, aph ^ 1, abort_flag, kWaitLimitNs)) { fail(3); break; }
-                tc_fence_after();
-                bool ok = true;
+            const int nb = tmem_batches(cf);
+            bool ok = true;
+            for (int64_t t = first; t < p.t_end && ok && !*abort_flag; t += gridDim.x) {
 #pragma unroll 1
-                for (int ei = 0; ei < cf.n; ++ei) {
+              for (int b0 = 0; b0 < nb * kTmemBatch && ok; b0 += kTmemBatch) {
+                if (!mbar_wait_bounded(acc_empty, aph ^ 1, abort_flag, kWaitLimitNs)) { fail(3); ok = false; break; }
+                tc_fence_after();
+                const int b1 = cf.n < b0 + kTmemBatch ? cf.n : b0 + kTmemBatch;
+#pragma unroll 1
+                for (int ei = b0; ei < b1; ++ei) {
                     if (!mbar_wait_bounded(&op_full[os], oph, abort_flag, kWaitLimitNs)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t a_s = smem_u32(op_ring + (size_t)os * C::kOpStageBytes);
@@ -347,7 +360,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
                         const uint64_t db = BBULK
                             ? smem_desc(a_s, C::kAHalfBytes, zero_s - a_s, kSwizzle128B)
                             : smem_desc(a_s + 2048u * k, C::kAHalfBytes, 1024, kSwizzle128B);
-                        tc_mma_f16(tmem_base + 128u * ei, da, db, idesc, k > 0 ? 1u : 0u);
+                        tc_mma_f16(tmem_base + 128u * (ei - b0), da, db, idesc, k > 0 ? 1u : 0u);
                     }
                     tc_commit(&op_empty[os]);
                     if (++os == C::kOpStages) { os = 0; oph ^= 1; }
@@ -355,6 +368,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
                 if (!ok) { fail(4); break; }
                 tc_commit(acc_full);
                 aph ^= 1;
+              }
             }
         }
     } else {
@@ -393,20 +407,29 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
             const int half = cgrp >> 1;             // which 64-column TMA box
             const int row = quarter * 32 + lane;
             const uint32_t t_lane = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(cgrp * 32);
+            const int nb = tmem_batches(cf);
             int ws = 0;
             uint32_t wph = 0, aph = 0;
             for (int64_t t = first; t < p.t_end; t += gridDim.x) {
                 if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
-                // 1) sum_e c_e * acc_e for this thread's row, 32 columns
-                bool ok = mbar_wait_bounded(acc_full, aph, abort_flag, kWaitLimitNs);
-                if (!__all_sync(0xffffffffu, ok)) { fail(5); break; }
-                aph ^= 1;
-                tc_fence_after();
+                // 1) sum_e c_e * acc_e for this thread's row, 32 columns,
+                //    one TMEM batch of up to four experts at a time
                 float tot[32];
-                epi_combine(t_lane, cf, tot);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(acc_empty);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) tot[i] = 0.f;
+                bool ok = true;
+#pragma unroll 1
+                for (int b0 = 0; b0 < nb * kTmemBatch; b0 += kTmemBatch) {
+                    ok = mbar_wait_bounded(acc_full, aph, abort_flag, kWaitLimitNs);
+                    if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                    aph ^= 1;
+                    tc_fence_after();
+                    epi_combine(t_lane, cf, b0, tot);
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(acc_empty);
+                }
+                if (!ok) { fail(5); break; }
 
                 // 2) W: smem (128B-swizzled rows of 64 columns) -> +dW -> smem
                 ok = mbar_wait_bounded(&w_full[ws], wph, abort_flag, kWaitLimitNs);

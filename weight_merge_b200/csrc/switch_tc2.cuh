@@ -95,8 +95,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc2_kernel(const TcParam
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epi_done + C::kWStages);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-    Coefs cf;
-    const int st = build_coefs(p.prev, p.cur, p.E, p.s, cf);
+    Coefs8 cf;
+    const int st = build_coefs(p.prev, p.cur, p.slots, p.E, p.s, cf);
     if (st != 0) {
         if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(p.status, st);
         return;
@@ -203,7 +203,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc2_kernel(const TcParam
                 const uint32_t bytes = (ti.rows ? C::kBBytes : 0u) + (load_a ? C::kAHalfBytes : 0u);
 #pragma unroll 1
                 for (int ei = 0; ei < cf.n; ++ei) {
-                    const int e = ei == 0 ? cf.e[0] : ei == 1 ? cf.e[1] : ei == 2 ? cf.e[2] : cf.e[3];
+                    const int e = coef_expert(cf, ei);
                     if (!mbar_wait_bounded(&op_empty[os], oph ^ 1, abort_flag, kWaitLimitNs)) { ok = false; break; }
                     uint8_t* a_dst = op_ring + (size_t)os * C::kOpStageBytes;
                     uint8_t* b_dst = a_dst + C::kAHalfBytes;
@@ -233,12 +233,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc2_kernel(const TcParam
             constexpr uint32_t idesc = instr_desc_bf16(kBlockRows, 128, /*B MN-major*/ 1);
             int os = 0;
             uint32_t oph = 0, aph = 0;
-            for (int64_t t = first; t < p.t_end && !*abort_flag; t += n_clusters) {
-                if (!mbar_wait_bounded(acc_empty, aph ^ 1, abort_flag, kWaitLimitNs)) { fail(3); break; }
-                tc_fence_after();
-                bool ok = true;
+            const int nb = tmem_batches(cf);
+            bool ok = true;
+            for (int64_t t = first; t < p.t_end && ok && !*abort_flag; t += n_clusters) {
 #pragma unroll 1
-                for (int ei = 0; ei < cf.n; ++ei) {
+              for (int b0 = 0; b0 < nb * kTmemBatch && ok; b0 += kTmemBatch) {
+                if (!mbar_wait_bounded(acc_empty, aph ^ 1, abort_flag, kWaitLimitNs)) { fail(3); ok = false; break; }
+                tc_fence_after();
+                const int b1 = cf.n < b0 + kTmemBatch ? cf.n : b0 + kTmemBatch;
+#pragma unroll 1
+                for (int ei = b0; ei < b1; ++ei) {
                     if (!mbar_wait_bounded(&op_full[os], oph, abort_flag, kWaitLimitNs)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t a_s = smem_u32(op_ring + (size_t)os * C::kOpStageBytes);
@@ -250,7 +254,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc2_kernel(const TcParam
                         // MMA B operand: KP x 64 A_e columns per CTA, N-major,
                         // 8-row K groups 1024 B apart (one swizzle atom wide)
                         const uint64_t db = smem_desc(a_s + 2048u * k, C::kAHalfBytes, 1024, kSwizzle128B);
-                        tc_mma_f16_pair(tmem_base + 128u * ei, da, db, idesc, k > 0 ? 1u : 0u);
+                        tc_mma_f16_pair(tmem_base + 128u * (ei - b0), da, db, idesc, k > 0 ? 1u : 0u);
                     }
                     tc_commit_pair(&op_empty[os], 0x3);
                     if (++os == C::kOpStages) { os = 0; oph ^= 1; }
@@ -258,6 +262,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc2_kernel(const TcParam
                 if (!ok) { fail(4); break; }
                 tc_commit_pair(acc_full, 0x3);
                 aph ^= 1;
+              }
             }
         }
     } else if (warp == 2) {
@@ -292,19 +297,28 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc2_kernel(const TcParam
         const int row = quarter * 32 + lane;
         const uint32_t t_lane = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(cgrp * 32);
         const uint32_t acc_empty0 = cluster_addr(acc_empty, 0);
+        const int nb = tmem_batches(cf);
         int ws = 0;
         uint32_t wph = 0, aph = 0;
         for (int64_t t = first; t < p.t_end; t += n_clusters) {
             if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
-            bool ok = mbar_wait_bounded(acc_full, aph, abort_flag, kWaitLimitNs);
-            if (!__all_sync(0xffffffffu, ok)) { fail(5); break; }
-            aph ^= 1;
-            tc_fence_after();
+            // one TMEM batch of up to four experts at a time
             float tot[32];
-            epi_combine(t_lane, cf, tot);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(acc_empty0);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) tot[i] = 0.f;
+            bool ok = true;
+#pragma unroll 1
+            for (int b0 = 0; b0 < nb * kTmemBatch; b0 += kTmemBatch) {
+                ok = mbar_wait_bounded(acc_full, aph, abort_flag, kWaitLimitNs);
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                aph ^= 1;
+                tc_fence_after();
+                epi_combine(t_lane, cf, b0, tot);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(acc_empty0);
+            }
+            if (!ok) { fail(5); break; }
 
             ok = mbar_wait_bounded(&w_full[ws], wph, abort_flag, kWaitLimitNs);
             if (!__all_sync(0xffffffffu, ok)) { fail(6); break; }
