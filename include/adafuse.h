@@ -254,6 +254,16 @@ ADAFUSE_API int adafuse_switch_topk_layers(adafuse_ctx* ctx, int32_t layer_begin
  * g_e B_e A_e).  INVALID_ARG without a registered base. */
 ADAFUSE_API int adafuse_rebase_topk(adafuse_ctx* ctx, const adafuse_route4* cur, void* stream);
 
+/* Test hook for the timeout path (no counterpart on the pages).  The next
+ * switch or re-base launched with a tensor-core kernel announces 16 bytes of
+ * operand transfers that never arrive on each CTA's first stage, so the MMA
+ * warp's bounded wait (1 s) runs out: the launch raises
+ * ADAFUSE_STATUS_TIMEOUT, every warp leaves through its bounded waits, TMEM is
+ * freed, no MMA completes and W is not written; the context stays usable.
+ * UNSUPPORTED_SHAPE when the context's kernel is ADAFUSE_KERNEL_MMA_SYNC (it
+ * has no waits).  Host-only; consumed by the next launch. */
+ADAFUSE_API int adafuse_debug_stall_next_switch(adafuse_ctx* ctx);
+
 /* Synchronise `stream`, read the device status word into *status, then
  * clear it.  Returns ADAFUSE_ERR_DEVICE_FAULT when the word was non-zero,
  * ADAFUSE_OK otherwise. */

@@ -163,3 +163,29 @@ def test_cuda_graph_capture_of_pregate_and_switch(kernel, r):
     for a, b in zip(m1.W, m2.W):
         assert torch.equal(a, b)
     assert torch.equal(r1[T - 1:T], cur)
+
+
+@pytest.mark.parametrize("kernel,r", [(TC, 8), (TC, 16), (TC2, 16), (TC2, 64)])
+def test_bounded_wait_timeout_reports_status_and_context_stays_usable(kernel, r):
+    """Failure detection without a GPU fault: the test hook makes each CTA's
+    first operand stage wait for 16 bytes that never arrive.  The MMA warp's
+    bounded wait (1 s) runs out, the launch raises ADAFUSE_STATUS_TIMEOUT and
+    every warp leaves through its own bounded waits before any MMA completes,
+    so W is untouched; the next switch on the same context is exact."""
+    cfg, m, sw = _model(kernel, seed=21, r=r)
+    assert sw.kernel == kernel
+    W0 = [bits(w) for w in m.W]
+    routes = make_routes(np.array([[0, 2], [3, 1]], np.int32),
+                         np.array([[0.7, 0.3], [0.6, 0.4]], np.float32))
+    Bnd.adafuse_debug_stall_next_switch(sw.ctx)
+    sw.switch(None, Bnd.Switcher.route_ptr(routes, 0), stream())
+    assert sw.status(stream()) == Bnd.ADAFUSE_STATUS_TIMEOUT
+    for w, w0 in zip(m.W, W0):
+        assert np.array_equal(bits(w), w0)
+    _switch_and_check(cfg, m, sw, routes, [(None, 0), (0, 1)])
+
+
+def test_stall_hook_is_refused_by_the_wait_free_kernel():
+    cfg, m, sw = _model(MMA, seed=22, r=8)
+    with pytest.raises(Bnd.AdafuseError):
+        Bnd.adafuse_debug_stall_next_switch(sw.ctx)

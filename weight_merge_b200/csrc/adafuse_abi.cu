@@ -36,6 +36,7 @@ struct adafuse_ctx {
     std::vector<PairDesc> h_pairs;  // host copy of d_pairs (re-base pointers are patched in)
     CUtensorMap* d_w0_maps = nullptr;  // 1 per pair on the re-base source W0
     bool has_base = false;
+    bool stall_next = false;  // test hook: the next tensor-core launch times out
     // pair kernel: 256 x 128 blocks, layer-major like the tile table
     TileEntry* d_blocks = nullptr;
     std::vector<int64_t> layer_block_begin;  // [n_layers + 1]
@@ -131,7 +132,7 @@ bool pair_eligible(const adafuse_ctx* c) { return c->tc_kp != 0 && c->rank != 8;
 int kp_class(int r) { return r <= 8 ? 8 : r <= 16 ? 16 : r <= 32 ? 32 : 64; }
 
 template <int KP, bool BBULK>
-cudaError_t launch_tc(const adafuse_ctx* c, int64_t t0, int64_t t1, const int32_t* prev,
+cudaError_t launch_tc(adafuse_ctx* c, int64_t t0, int64_t t1, const int32_t* prev,
                       const int32_t* cur, int slots, cudaStream_t s, bool rebase) {
     TcParams prm;
     prm.pairs = c->d_pairs;
@@ -147,6 +148,8 @@ cudaError_t launch_tc(const adafuse_ctx* c, int64_t t0, int64_t t1, const int32_
     prm.status = c->d_status;
     prm.rebase = rebase ? 1 : 0;
     prm.w0_maps = c->d_w0_maps;
+    prm.stall = c->stall_next ? 1 : 0;
+    c->stall_next = false;
     return launch_switch_tc<KP, BBULK>(prm, c->device, c->sm_count, s);
 }
 
@@ -174,6 +177,8 @@ cudaError_t launch_tc2(adafuse_ctx* c, int64_t b0, int64_t b1, const int32_t* pr
     prm.status = c->d_status;
     prm.rebase = rebase ? 1 : 0;
     prm.w0_maps = c->d_w0_maps;
+    prm.stall = c->stall_next ? 1 : 0;
+    c->stall_next = false;
     return launch_switch_tc2<KP>(prm, c->pair_clusters, s);
 }
 
@@ -624,6 +629,13 @@ int adafuse_switch_topk(adafuse_ctx* ctx, const adafuse_route4* prev, const adaf
 int adafuse_rebase_topk(adafuse_ctx* ctx, const adafuse_route4* cur, void* stream) {
     if (ctx == nullptr || !ctx->has_base) return ADAFUSE_ERR_INVALID_ARG;
     return launch_switch(ctx, 0, ctx->n_layers, nullptr, cur, 4, stream, true);
+}
+
+int adafuse_debug_stall_next_switch(adafuse_ctx* ctx) {
+    if (ctx == nullptr) return ADAFUSE_ERR_INVALID_ARG;
+    if (adafuse_get_switch_kernel(ctx) == ADAFUSE_KERNEL_MMA_SYNC) return ADAFUSE_ERR_UNSUPPORTED_SHAPE;
+    ctx->stall_next = true;
+    return ADAFUSE_OK;
 }
 
 int adafuse_get_device_status(adafuse_ctx* ctx, void* stream, int32_t* status) {

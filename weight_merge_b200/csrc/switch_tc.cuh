@@ -42,6 +42,7 @@ constexpr int kTcEpiThreads = 512;         // warps 4..19
 constexpr uint32_t kWTileBytes = 128 * 128 * 2;
 constexpr uint32_t kWBoxBytes = kWTileBytes / 2;   // 128 rows x 64 cols
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
+constexpr uint32_t kStallBytes = 16;
 
 // KP: per-expert contraction depth (rank padded to 16, 32 or 64).
 // BBULK: rank 8.  Its B rows (128 x 8) are one contiguous 2 KB block already in
@@ -91,6 +92,10 @@ struct TcParams {
     // a tile is written even when no expert is selected (it copies W0).
     int rebase;
     const CUtensorMap* w0_maps;
+    // test hook: each CTA's first operand stage announces kStallBytes more
+    // than its loads deliver, so the MMA warp's bounded wait runs out and the
+    // launch ends through the timeout path before any MMA completes
+    int stall;
 };
 
 // Tile entries are fetched one iteration ahead (the loops below keep the next
@@ -305,10 +310,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
                         // rows past the weight's end are not fetched (their
                         // products only reach accumulator rows never stored)
                         const uint32_t bbytes = (uint32_t)out_rows * 16u;
-                        mbar_arrive_expect_tx(&op_full[os], bbytes + (second ? 2 : 1) * C::kAHalfBytes);
+                        mbar_arrive_expect_tx(&op_full[os], bbytes + (second ? 2 : 1) * C::kAHalfBytes +
+                                                                (p.stall && t == first && ei == 0 ? kStallBytes : 0u));
                         bulk_load(b_dst, Bbase + ((size_t)e * out + row0) * 8, bbytes, &op_full[os]);
                     } else {
-                        mbar_arrive_expect_tx(&op_full[os], C::kBBytes + (second ? 2 : 1) * C::kAHalfBytes);
+                        mbar_arrive_expect_tx(&op_full[os], C::kBBytes + (second ? 2 : 1) * C::kAHalfBytes +
+                                                                (p.stall && t == first && ei == 0 ? kStallBytes : 0u));
                         tma_load_3d(b_dst, mB, 0, row0, e, &op_full[os]);
                     }
                     tma_load_3d(a_dst, mA, col0, 0, e, &op_full[os]);
