@@ -305,3 +305,59 @@ def test_switch_topk_llama2_7b_shape_sampled():
     sw.close()
     del model
     torch.cuda.empty_cache()
+
+
+# --------------------------------------------------------------------------
+# limits: the largest expert count, odd sizes, misaligned routes
+
+@pytest.mark.parametrize("kernel", [MMA, TC, TC2])
+def test_switch_topk_sixty_four_experts_rank_64(kernel):
+    """E = 64 (the largest expert count) at rank 64: the TMA maps span the
+    whole stacked adapter tensors; experts come from the far end too."""
+    cfg = wl.custom("e64", 1, [("a", 264, 136), ("b", 128, 392)], n_experts=64, rank=64,
+                    alpha=128.0, n_tokens=3, d=136)
+    model = wl.make_model(cfg, device="cuda", seed=64)
+    sw = switcher(model, kernel)
+    idx = np.array([[63, 0, 31, 62], [1, 63, 40, 2], [62, 61, -1, -1]], np.int32)
+    gate = np.array([[0.4, 0.3, 0.2, 0.1], [0.5, 0.2, 0.2, 0.1], [0.6, 0.4, 0, 0]], np.float32)
+    routes = make_routes4(idx, gate)
+    A_h, B_h = [bits(a) for a in model.A], [bits(b) for b in model.B]
+    _lockstep(sw, model, routes, [(None, 0), (0, 1), (1, 2)], A_h, B_h)
+
+
+@pytest.mark.parametrize("T,d,E,k", [(5, 4100, 64, 4), (130, 1028, 64, 3), (1, 12, 5, 4)])
+def test_pregate_topk_odd_sizes_and_many_experts(T, d, E, k):
+    cfg = wl.custom("p", 1, [("q", 8, 8)], n_experts=E, rank=8, alpha=16, n_tokens=T, d=d)
+    sw = switcher(wl.make_model(cfg, device="cuda", seed=E))
+    g = torch.Generator(device="cuda").manual_seed(300 + d)
+    h = torch.randn((T, d), generator=g, device="cuda")
+    Wr = torch.randn((d, E), generator=g, device="cuda") * 0.05
+    routes = torch.zeros((T, 8), dtype=torch.int32, device="cuda")
+    sw.pregate_topk(h, Wr, k, routes, stream())
+    torch.cuda.synchronize()
+    got = routes4_to_np(routes)
+    h_np, Wr_np = h.cpu().numpy(), Wr.cpu().numpy()
+    idx_ref, gate_ref, z = oracle.pregate_topk(h_np, Wr_np, k, return_logits=True)
+    amb = pregate_topk_consistent(got[:, :k], idx_ref, z, h_np, Wr_np)
+    assert len(amb) <= max(1, T // 50)
+    match = np.all(got[:, :k] == idx_ref, axis=1)
+    np.testing.assert_allclose(got[match, 4:4 + k].view(np.float32), gate_ref[match],
+                               rtol=GATE_RTOL, atol=1e-30)
+
+
+def test_topk_entry_points_refuse_misaligned_routes():
+    model = _small(seed=12, r=8)
+    sw = switcher(model)
+    buf = torch.zeros((4, 8), dtype=torch.int32, device="cuda")
+    bad = buf.data_ptr() + 4          # not 16-byte aligned
+    good = buf.data_ptr()
+    with pytest.raises(Bnd.AdafuseError):
+        sw.switch_topk(bad, good, stream())
+    with pytest.raises(Bnd.AdafuseError):
+        sw.switch_topk(good, bad, stream())
+    h = torch.zeros((1, 384), device="cuda")
+    with pytest.raises(Bnd.AdafuseError):
+        Bnd.adafuse_pregate_topk(sw.ctx, h.data_ptr(), 1, 384, model.Wr.data_ptr(), 2, bad, stream())
+    sw.switch_topk_layers(0, 0, good, good, stream())   # an empty layer range is a no-op
+    with pytest.raises(Bnd.AdafuseError):
+        sw.switch_topk_layers(2, 2, good, good, stream())
