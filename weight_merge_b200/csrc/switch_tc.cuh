@@ -347,8 +347,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
                 const int b1 = cf.n < b0 + kTmemBatch ? cf.n : b0 + kTmemBatch;
 #pragma unroll 1
                 for (int ei = b0; ei < b1; ++ei) {
+                    // TMA's complete_tx on the mbarrier orders the operand
+                    // bytes before the MMA's shared-memory reads: no tcgen05 fence
                     if (!mbar_wait_bounded(&op_full[os], oph, abort_flag, kWaitLimitNs)) { ok = false; break; }
-                    tc_fence_after();
                     const uint32_t a_s = smem_u32(op_ring + (size_t)os * C::kOpStageBytes);
                     const uint32_t b_s = a_s + C::kABytes;
 #pragma unroll
