@@ -41,6 +41,8 @@
  * in place for the life of the context, and must not write W while a switch
  * on it is in flight.  The library owns the context, its device-side
  * segment table and its device status word.  The library keeps no copy of W.
+ * For ranks below 8 it keeps a zero-padded copy of every B (see
+ * adafuse_refresh_adapters).
  *
  * Errors: every call returns ADAFUSE_OK (0) or a negative code.  Calls that
  * take a stream are asynchronous with respect to the host; host-side
@@ -82,10 +84,10 @@ extern "C" {
                                              (the switch is then incomplete) */
 
 /* ---- switch kernel variants (adafuse_set_switch_kernel) ------------------ */
-#define ADAFUSE_KERNEL_AUTO      0  /* rank 8: TCGEN05; other multiples of 8: TCGEN05_PAIR;
+#define ADAFUSE_KERNEL_AUTO      0  /* rank <= 8: TCGEN05; other multiples of 8: TCGEN05_PAIR;
                                        any other rank: MMA_SYNC */
 #define ADAFUSE_KERNEL_MMA_SYNC  1  /* register-streaming kernel, any rank in [1, 64] */
-#define ADAFUSE_KERNEL_TCGEN05   2  /* TMA + tcgen05/TMEM kernel, rank a multiple of 8 */
+#define ADAFUSE_KERNEL_TCGEN05   2  /* TMA + tcgen05/TMEM kernel, rank <= 8 or a multiple of 8 */
 #define ADAFUSE_KERNEL_TCGEN05_PAIR 3 /* the same on CTA pairs (tcgen05 cta_group::2, 256 x 128
                                          W blocks), rank a multiple of 8 */
 
@@ -188,9 +190,9 @@ ADAFUSE_API int adafuse_switch_batch_layers(adafuse_ctx* ctx, int32_t layer_begi
 
 /* Choose the kernel adafuse_switch launches for this context (default
  * ADAFUSE_KERNEL_AUTO).  All compute the same update to within the
- * documented rounding; ADAFUSE_KERNEL_TCGEN05 and ADAFUSE_KERNEL_TCGEN05_PAIR
- * need rank % 8 == 0 and return UNSUPPORTED_SHAPE otherwise.  Host-only, no
- * device work. */
+ * documented rounding; ADAFUSE_KERNEL_TCGEN05 needs rank <= 8 or a multiple
+ * of 8, ADAFUSE_KERNEL_TCGEN05_PAIR a multiple of 8 above 8; both return
+ * UNSUPPORTED_SHAPE otherwise.  Host-only, no device work. */
 ADAFUSE_API int adafuse_set_switch_kernel(adafuse_ctx* ctx, int kernel);
 
 /* The kernel adafuse_switch will launch (ADAFUSE_KERNEL_MMA_SYNC,
@@ -253,6 +255,14 @@ ADAFUSE_API int adafuse_switch_topk_layers(adafuse_ctx* ctx, int32_t layer_begin
 /* As adafuse_rebase with a top-k route: W <- bf16_rne(W0 + s*sum_{e in cur}
  * g_e B_e A_e).  INVALID_ARG without a registered base. */
 ADAFUSE_API int adafuse_rebase_topk(adafuse_ctx* ctx, const adafuse_route4* cur, void* stream);
+
+/* Ranks below 8 only (a no-op otherwise): the tensor-core path reads B
+ * through a copy whose rows are zero-padded to 8 (B rows of 2*rank bytes are
+ * not a legal TMA stride).  adafuse_create takes that copy; after changing
+ * the contents of any B of the context, call this before the next switch.
+ * It enqueues the copies on `stream`.  The copy costs 8/rank times the bytes
+ * of the B tensors in device memory. */
+ADAFUSE_API int adafuse_refresh_adapters(adafuse_ctx* ctx, void* stream);
 
 /* Test hook for the timeout path (no counterpart on the pages).  The next
  * switch or re-base launched with a tensor-core kernel announces 16 bytes of

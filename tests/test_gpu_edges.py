@@ -13,14 +13,15 @@ import oracle
 from weight_merge_b200 import binding as Bnd
 from weight_merge_b200 import workloads as wl
 
-from .util import bits, check_switch_rows, make_routes, route_tuple, routes_to_np
+from .util import (bf16_to_f64, bits, check_switch_rows, fp32_accum_gamma, make_routes,
+                   route_tuple, routes_to_np, ulp_dist)
 
 pytestmark = pytest.mark.gpu
 
 MMA, TC, TC2 = (Bnd.ADAFUSE_KERNEL_MMA_SYNC, Bnd.ADAFUSE_KERNEL_TCGEN05,
                 Bnd.ADAFUSE_KERNEL_TCGEN05_PAIR)
 # each kernel at a rank it takes
-KERNEL_RANKS = [(MMA, 8), (TC, 8), (TC2, 16)]
+KERNEL_RANKS = [(MMA, 8), (TC, 8), (TC, 4), (TC2, 16)]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -84,17 +85,25 @@ def test_subnormal_results(kernel, r):
 @pytest.mark.parametrize("kernel,r", KERNEL_RANKS)
 def test_overflow_to_infinity(kernel, r):
     """W at the largest bf16 magnitudes plus a same-signed dW rounds to +-inf,
-    as the oracle's round-to-nearest-even does."""
+    as the oracle's round-to-nearest-even does.
+
+    Under round-to-nearest-even a magnitude rounds to inf from
+    2^128 - 2^119 up (half a step above the largest finite bf16, the tie
+    going to the even pattern, inf).  Where the exact fp64 value lies within
+    the fp32 accumulation bound of that threshold either side is a correct
+    rounding of an fp32 sum, so there the 1-step parity bar decides; every
+    other element must land on the oracle's side of it."""
     cfg, m, sw = _model(kernel, seed=4, r=r)
     with torch.no_grad():
         for w in m.W:
             w.copy_(torch.where(w >= 0, 3.3895e38, -3.3895e38).to(torch.bfloat16))
-        # |B| ~ 2e36, |A| ~ 0.05: dW ~ 1e36 > half a bf16 step at 3.39e38 (6.6e35),
-        # positive everywhere, while every fp32 partial stays finite
+        # |B| ~ 2e36, |A| ~ 0.05: dW ~ r * 1.3e35, against half a bf16 step at
+        # 3.39e38 (6.6e35); positive everywhere, every fp32 partial finite
         for b in m.B:
             b.abs_().mul_(3e38)
         for a in m.A:
             a.abs_()
+    Bnd.adafuse_refresh_adapters(sw.ctx, stream())   # B changed after create (rank < 8 copy)
     routes = make_routes(np.array([[0, 1]], np.int32), np.array([[0.5, 0.5]], np.float32))
     before = [bits(w) for w in m.W]
     sw.switch(None, Bnd.Switcher.route_ptr(routes, 0), stream())
@@ -102,15 +111,24 @@ def test_overflow_to_infinity(kernel, r):
     A_h = [bits(a) for a in m.A]
     B_h = [bits(b) for b in m.B]
     r_np = routes_to_np(routes)
+    thr = 2.0 ** 128 - 2.0 ** 119
+    gamma = fp32_accum_gamma(r, 2)
     for i, w in enumerate(m.W):
         got = bits(w)
-        want = oracle.switch(before[i], A_h[i], B_h[i], cfg.scale, None, route_tuple(r_np, 0))
-        inf_want = (want & 0x7FFF) == 0x7F80
-        assert inf_want.sum() > 0                       # some really overflow
-        assert np.array_equal(got[inf_want], want[inf_want])
-        # negative W moves away from the overflow and stays finite
-        fin = ~inf_want
-        assert np.all((got[fin] & 0x7F80) != 0x7F80)
+        want, exact = oracle.switch(before[i], A_h[i], B_h[i], cfg.scale, None,
+                                    route_tuple(r_np, 0), exact=True)
+        M = np.abs(bf16_to_f64(before[i]))
+        for e, g in zip(*route_tuple(r_np, 0)):
+            M += cfg.scale * float(g) * (np.abs(bf16_to_f64(B_h[i][e])) @ np.abs(bf16_to_f64(A_h[i][e])))
+        margin = gamma * M
+        over = np.abs(exact) >= thr + margin
+        under = np.abs(exact) < thr - margin
+        is_inf = (got & 0x7FFF) == 0x7F80
+        assert over.sum() > 0                           # some really overflow
+        assert np.array_equal(got[over], want[over])    # to inf of the right sign
+        assert not is_inf[under].any()                  # the rest stays finite
+        assert not is_inf[(before[i] & 0x8000) != 0].any()   # negative W moves away
+        assert ulp_dist(got, want).max() <= 1
 
 
 def test_pregate_empty_batch_is_a_noop():
@@ -189,3 +207,20 @@ def test_stall_hook_is_refused_by_the_wait_free_kernel():
     cfg, m, sw = _model(MMA, seed=22, r=8)
     with pytest.raises(Bnd.AdafuseError):
         Bnd.adafuse_debug_stall_next_switch(sw.ctx)
+
+
+@pytest.mark.parametrize("r", [1, 4, 7])
+def test_ranks_below_8_read_a_padded_copy_of_b_refreshed_on_request(r):
+    """Below rank 8 the tensor-core path reads B through the context's
+    zero-padded copy.  After the caller changes B, adafuse_refresh_adapters
+    brings the copy up to date and the switch matches the oracle on the new B."""
+    cfg, m, sw = _model(TC, seed=30 + r, r=r)
+    assert sw.kernel == TC
+    routes = make_routes(np.array([[0, 2], [3, 1]], np.int32),
+                         np.array([[0.7, 0.3], [0.6, 0.4]], np.float32))
+    _switch_and_check(cfg, m, sw, routes, [(None, 0)])
+    with torch.no_grad():
+        for b in m.B:
+            b.mul_(-1.5)
+    Bnd.adafuse_refresh_adapters(sw.ctx, stream())
+    _switch_and_check(cfg, m, sw, routes, [(0, 1), (1, None)])

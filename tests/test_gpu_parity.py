@@ -54,9 +54,9 @@ def make_switcher(model: wl.Model, kernel: int = Bnd.ADAFUSE_KERNEL_AUTO) -> Bnd
 
 
 def kernels_for(rank):
-    if rank % 8 != 0:
-        return [MMA]
-    return [MMA, TC] if rank == 8 else [MMA, TC, TC2]
+    if rank <= 8:
+        return [MMA, TC]
+    return [MMA, TC, TC2] if rank % 8 == 0 else [MMA]
 
 
 # (kernel, rank) for the small-model tests: each kernel at a rank it takes
@@ -361,14 +361,14 @@ def _full_size_case(name, n_switches, full_first=True, kernel=Bnd.ADAFUSE_KERNEL
 
 
 def test_auto_picks_tensor_cores_when_rank_allows():
-    for r, want in [(4, MMA), (8, TC), (12, MMA), (16, TC2), (24, TC2), (64, TC2)]:
+    for r, want in [(1, TC), (4, TC), (7, TC), (8, TC), (12, MMA), (16, TC2), (24, TC2), (64, TC2)]:
         cfg = wl.custom("k", 1, [("q", 64, 64)], n_experts=2, rank=r, alpha=2.0 * r, n_tokens=1)
         sw = make_switcher(wl.make_model(cfg, device="cuda"))
         assert sw.kernel == want
         if want == MMA:
             with pytest.raises(Bnd.AdafuseError):
                 sw.set_kernel(TC)
-        if r == 8:
+        if r <= 8:
             with pytest.raises(Bnd.AdafuseError):
                 sw.set_kernel(TC2)
 

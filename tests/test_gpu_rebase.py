@@ -58,7 +58,8 @@ def _check_against_oracle(cfg, m, W0, route, A_h, B_h):
 
 @pytest.mark.parametrize("E,r,kernel", [(3, 3, MMA), (4, 8, MMA), (4, 8, TC), (5, 16, TC),
                                         (3, 24, MMA), (4, 32, TC), (6, 64, TC), (5, 16, TC2),
-                                        (3, 24, TC2), (4, 32, TC2), (6, 64, TC2)])
+                                        (3, 24, TC2), (4, 32, TC2), (6, 64, TC2), (3, 3, TC),
+                                        (4, 4, TC)])
 def test_rebase_matches_oracle_and_does_not_accumulate(E, r, kernel):
     cfg, m, sw, W0 = _setup(E, r, kernel, seed=31 * r + E)
     W0_bits = [bits(w) for w in W0]

@@ -47,9 +47,9 @@ def switcher(model, kernel=Bnd.ADAFUSE_KERNEL_AUTO):
 
 
 def kernels_for(rank):
-    if rank % 8 != 0:
-        return [MMA]
-    return [MMA, TC] if rank == 8 else [MMA, TC, TC2]
+    if rank <= 8:
+        return [MMA, TC]
+    return [MMA, TC, TC2] if rank % 8 == 0 else [MMA]
 
 
 # --------------------------------------------------------------------------
@@ -198,7 +198,7 @@ def _small(seed=3, E=8, r=16):
     return wl.make_model(cfg, device="cuda", seed=seed)
 
 
-KERNEL_RANKS = [(MMA, 8), (TC, 8), (TC, 16), (TC2, 16)]
+KERNEL_RANKS = [(MMA, 8), (TC, 8), (TC, 4), (TC, 16), (TC2, 16)]
 
 
 @pytest.mark.parametrize("kernel,r", KERNEL_RANKS)

@@ -95,6 +95,7 @@ def lib() -> ctypes.CDLL:
         "adafuse_switch_topk_layers": ([P, i32, i32, P, P, P], ctypes.c_int),
         "adafuse_rebase_topk": ([P, P, P], ctypes.c_int),
         "adafuse_debug_stall_next_switch": ([P], ctypes.c_int),
+        "adafuse_refresh_adapters": ([P, P], ctypes.c_int),
         "adafuse_segment_table": ([ctypes.POINTER(Desc), P, i64, ctypes.POINTER(i64)], ctypes.c_int),
         "adafuse_tile_size": ([], ctypes.c_int),
         "adafuse_strerror": ([ctypes.c_int], ctypes.c_char_p),
@@ -189,6 +190,10 @@ def adafuse_switch_topk_layers(ctx: int, layer_begin: int, n_layers: int, prev: 
 
 def adafuse_rebase_topk(ctx: int, cur: Optional[int], stream: int = 0) -> None:
     _check(lib().adafuse_rebase_topk(ctx, cur or None, stream or None), "adafuse_rebase_topk")
+
+
+def adafuse_refresh_adapters(ctx: int, stream: int = 0) -> None:
+    _check(lib().adafuse_refresh_adapters(ctx, stream or None), "adafuse_refresh_adapters")
 
 
 def adafuse_debug_stall_next_switch(ctx: int) -> None:

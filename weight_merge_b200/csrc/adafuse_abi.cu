@@ -39,6 +39,7 @@ struct adafuse_ctx {
     bool stall_next = false;  // test hook: the next tensor-core launch times out
     // pair kernel: 256 x 128 blocks, layer-major like the tile table
     TileEntry* d_blocks = nullptr;
+    uint16_t* d_bpad = nullptr;              // rank < 8: B with rows zero-padded to 8
     std::vector<int64_t> layer_block_begin;  // [n_layers + 1]
     int pair_clusters = 0;                   // co-resident CTA pairs (0 = not queried yet)
 };
@@ -127,7 +128,20 @@ int64_t walk_blocks(const adafuse_desc* d, Emit&& emit) {
 
 // The pair kernel takes the tensor-core kernel's ranks except 8 (whose A
 // tensor maps fetch exactly 8 rows for the single-CTA kernel's layout).
-bool pair_eligible(const adafuse_ctx* c) { return c->tc_kp != 0 && c->rank != 8; }
+bool pair_eligible(const adafuse_ctx* c) { return c->tc_kp != 0 && c->rank > 8; }
+
+// Rank < 8: copy every B [E, out, r] into its [E, out, 8] zero-padded slot
+// (the padding columns are zeroed once, at create).
+cudaError_t copy_padded_b(const adafuse_ctx* c, cudaStream_t s) {
+    for (const PairDesc& pd : c->h_pairs) {
+        const size_t rows = (size_t)c->n_experts * (size_t)pd.out;
+        const cudaError_t e = cudaMemcpy2DAsync(const_cast<uint16_t*>(pd.Bk), 16, pd.B,
+                                                (size_t)c->rank * 2, (size_t)c->rank * 2, rows,
+                                                cudaMemcpyDeviceToDevice, s);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
 
 int kp_class(int r) { return r <= 8 ? 8 : r <= 16 ? 16 : r <= 32 ? 32 : 64; }
 
@@ -257,6 +271,7 @@ int adafuse_create(adafuse_ctx** out, const adafuse_desc* desc, int device) {
         pairs[i].W0 = nullptr;
         pairs[i].A = static_cast<const uint16_t*>(t.A);
         pairs[i].B = static_cast<const uint16_t*>(t.B);
+        pairs[i].Bk = pairs[i].B;
         pairs[i].out = (int32_t)t.out;
         pairs[i].in = (int32_t)t.in;
         pairs[i].layer = (int32_t)(i / desc->n_targets);
@@ -293,9 +308,28 @@ int adafuse_create(adafuse_ctx** out, const adafuse_desc* desc, int device) {
         cudaFree(c->d_status);
         cudaFree(c->d_maps);
         cudaFree(c->d_blocks);
+        cudaFree(c->d_bpad);
         delete c;
         return err == cudaErrorMemoryAllocation ? ADAFUSE_ERR_OUT_OF_MEMORY : cuda_fail(err, what);
     };
+    // ranks below 8: the tensor-core path reads B through a copy with 16-byte
+    // rows (a legal TMA stride), zero-padded past the rank
+    if (desc->rank < 8 && tc_kp_for(desc->rank) != 0) {
+        size_t total = 0;
+        for (const PairDesc& pd : pairs) total += (size_t)desc->n_experts * (size_t)pd.out * 8;
+        if ((e = cudaMalloc(&c->d_bpad, total * 2)) != cudaSuccess)
+            return fail(e, "cudaMalloc(padded B)");
+        if ((e = cudaMemset(c->d_bpad, 0, total * 2)) != cudaSuccess)
+            return fail(e, "cudaMemset(padded B)");
+        size_t off = 0;
+        for (PairDesc& pd : pairs) {
+            pd.Bk = c->d_bpad + off;
+            off += (size_t)desc->n_experts * (size_t)pd.out * 8;
+        }
+        c->h_pairs = pairs;
+        if ((e = copy_padded_b(c, nullptr)) != cudaSuccess) return fail(e, "cudaMemcpy2D(padded B)");
+        if ((e = cudaDeviceSynchronize()) != cudaSuccess) return fail(e, "padded B");
+    }
     if ((e = cudaMalloc(&c->d_pairs, sizeof(PairDesc) * pairs.size())) != cudaSuccess)
         return fail(e, "cudaMalloc(pairs)");
     if ((e = cudaMalloc(&c->d_tiles, sizeof(TileEntry) * tiles.size())) != cudaSuccess)
@@ -373,6 +407,7 @@ int adafuse_destroy(adafuse_ctx* ctx) {
     cudaFree(ctx->d_maps);
     cudaFree(ctx->d_w0_maps);
     cudaFree(ctx->d_blocks);
+    cudaFree(ctx->d_bpad);
     delete ctx;
     return ADAFUSE_OK;
 }
@@ -508,7 +543,7 @@ int launch_switch(adafuse_ctx* ctx, int32_t layer_begin, int32_t n_layers,
     }
     if (kind == ADAFUSE_KERNEL_TCGEN05) {
         cudaError_t e = cudaSuccess;
-        if (ctx->rank == 8)
+        if (ctx->rank <= 8)
             e = launch_tc<16, true>(ctx, t0, t1, prev, cur, slots, s, rebase);
         else if (ctx->tc_kp == 16)
             e = launch_tc<16, false>(ctx, t0, t1, prev, cur, slots, s, rebase);
@@ -629,6 +664,15 @@ int adafuse_switch_topk(adafuse_ctx* ctx, const adafuse_route4* prev, const adaf
 int adafuse_rebase_topk(adafuse_ctx* ctx, const adafuse_route4* cur, void* stream) {
     if (ctx == nullptr || !ctx->has_base) return ADAFUSE_ERR_INVALID_ARG;
     return launch_switch(ctx, 0, ctx->n_layers, nullptr, cur, 4, stream, true);
+}
+
+int adafuse_refresh_adapters(adafuse_ctx* ctx, void* stream) {
+    if (ctx == nullptr) return ADAFUSE_ERR_INVALID_ARG;
+    if (ctx->d_bpad == nullptr) return ADAFUSE_OK;
+    DeviceGuard guard(ctx->device);
+    if (!guard.ok) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
+    const cudaError_t e = copy_padded_b(ctx, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ADAFUSE_OK : cuda_fail(e, "cudaMemcpy2D(padded B)");
 }
 
 int adafuse_debug_stall_next_switch(adafuse_ctx* ctx) {

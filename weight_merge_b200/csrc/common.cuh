@@ -18,6 +18,8 @@ struct PairDesc {
     const uint16_t* A;   // [E, r, in]
     const uint16_t* B;   // [E, out, r]
     const uint16_t* W0;  // [out, in] pristine base for the re-base switch (or null)
+    const uint16_t* Bk;  // [E, out, 8] B with 16-byte rows for the rank <= 8 tensor-core
+                         // path: B itself at rank 8, a zero-padded copy below
     int32_t out;
     int32_t in;
     int32_t layer;

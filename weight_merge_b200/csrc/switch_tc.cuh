@@ -45,7 +45,8 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
 constexpr uint32_t kStallBytes = 16;
 
 // KP: per-expert contraction depth (rank padded to 16, 32 or 64).
-// BBULK: rank 8.  Its B rows (128 x 8) are one contiguous 2 KB block already in
+// BBULK: rank <= 8.  Its B rows (128 x 8, from B itself at rank 8 or from the
+// context's zero-padded copy below) are one contiguous 2 KB block already in
 // the plain core-matrix layout, fetched with one bulk copy; its A columns are
 // an 8-row TMA box per 64-column half, and the MMA's second 8-deep K group
 // reads a shared zero block instead (through the descriptor's K-group stride),
@@ -296,7 +297,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
                 if constexpr (BBULK) {
                     const PairDesc& pd = p.pairs[pair];
                     out = pd.out;
-                    Bbase = pd.B;
+                    Bbase = pd.Bk;
                     out_rows = out - row0 < 128 ? out - row0 : 128;
                 }
                 bool ok = true;

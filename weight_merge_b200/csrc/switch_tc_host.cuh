@@ -5,14 +5,21 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <cstring>
+
 #include "common.cuh"
 #include "switch_tc.cuh"
 #include "switch_tc2.cuh"
 
 namespace adafuse {
 
-// The tensor-core kernel needs TMA-legal strides (rank a multiple of 8).
-inline int tc_kp_for(int r) { return (r % 8 != 0 || r > 64) ? 0 : r <= 16 ? 16 : r <= 32 ? 32 : 64; }
+// The tensor-core kernel needs TMA-legal strides: rank a multiple of 8, or
+// below 8 with B read from a copy whose rows are padded to 8.
+inline int tc_kp_for(int r) {
+    if (r < 1 || r > 64) return 0;
+    if (r < 8) return 16;
+    return r % 8 != 0 ? 0 : r <= 16 ? 16 : r <= 32 ? 32 : 64;
+}
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -52,13 +59,19 @@ inline bool encode_pair_maps(EncodeTiledFn enc, const PairDesc& pd, int E, int r
     {
         const cuuint64_t dims[3] = {(cuuint64_t)pd.in, (cuuint64_t)r, (cuuint64_t)E};
         const cuuint64_t strides[2] = {(cuuint64_t)pd.in * 2, (cuuint64_t)pd.in * r * 2};
-        // rank 8 fetches exactly its 8 rows; other ranks a KP-row box whose
-        // rows past r read as zero
-        const cuuint32_t box[3] = {64, (cuuint32_t)(r == 8 ? 8 : kp), 1};
+        // ranks up to 8 fetch an 8-row box, other ranks a KP-row box; rows
+        // past r read as zero
+        const cuuint32_t box[3] = {64, (cuuint32_t)(r <= 8 ? 8 : kp), 1};
         if (enc(&out[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, (void*)pd.A, dims, strides, box,
                 ones, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                 CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return false;
+    }
+    if (r < 8) {
+        // B rows of 2r bytes are not a legal TMA stride; the rank <= 8 path
+        // bulk-copies the padded rows instead and never uses this map
+        std::memset(&out[2], 0, sizeof(CUtensorMap));
+        return true;
     }
     {
         const cuuint64_t dims[3] = {(cuuint64_t)r, (cuuint64_t)pd.out, (cuuint64_t)E};
