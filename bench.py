@@ -60,6 +60,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-torch-baseline", action="store_true",
                     help="skip the unfused per-weight torch addmm_ context figure")
+    ap.add_argument("--no-layerwise", action="store_true",
+                    help="skip the per-layer-launch CUDA graph context figure")
     return ap.parse_args()
 
 
@@ -348,6 +350,51 @@ def torch_addmm_baseline(model, cfg, r_np, t_prev, t_cur, stream, reps=5):
                     "context only"}
 
 
+def layerwise_graph(sw, cfg, routes, r_np, t_from, stream, reps=6):
+    """The same switch issued as one launch per layer, the granularity at which
+    a decode forward can run layer l while later layers still switch (the
+    pages' in-place update pipelined behind the forward pass).  Two CUDA
+    graphs, t_from -> x and x -> t_from, are captured once and replayed in
+    turn, so W ends on the route it started from.  Context for the cost of
+    that granularity against the single launch; the forward itself is not
+    part of this library."""
+    import numpy as np
+    import torch
+    from weight_merge_b200 import binding as B
+
+    x = next((t for t in range(routes.shape[0]) if not np.array_equal(r_np[t], r_np[t_from])),
+             None)
+    if x is None:
+        return None
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    graphs = []
+    for a, b in ((t_from, x), (x, t_from)):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g, stream=side):
+                for layer in range(cfg.n_layers):
+                    sw.switch_layers(layer, 1, B.Switcher.route_ptr(routes, a),
+                                     B.Switcher.route_ptr(routes, b), side.cuda_stream)
+        graphs.append(g)
+    stream.wait_stream(side)
+    for g in graphs:
+        g.replay()
+    torch.cuda.synchronize()
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(2 * reps)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(2 * reps)]
+    for i in range(2 * reps):
+        ev0[i].record(stream)
+        graphs[i % 2].replay()
+        ev1[i].record(stream)
+    torch.cuda.synchronize()
+    ms = statistics.median(a.elapsed_time(b) for a, b in zip(ev0, ev1))
+    del graphs
+    return {"launches_per_switch": cfg.n_layers, "ms": round(ms, 4),
+            "hbm_gbs": round(cfg.w_bytes_per_switch() / (ms / 1e3) / 1e9, 1),
+            "replays": 2 * reps}
+
+
 def reduce_over_ranks(total_ms, n_units, world, device="cpu"):
     """Whole-job timing: the slowest rank's device time and the units (real
     switches) all ranks processed.  Every rank takes the same collective
@@ -486,6 +533,7 @@ def run_ours(args):
 
     # e2e through the public API with host buffers
     e2e = None
+    last_t = prev_t                  # the route W currently carries
     if not args.no_e2e:
         h_host = h.cpu().pin_memory()
         r_host = torch.zeros((1, routes.shape[1]), dtype=torch.int32).pin_memory()
@@ -503,6 +551,7 @@ def run_ours(args):
             do_switch(pe, t)
             r_host.copy_(routes[t:t + 1], non_blocking=True)
             pe = t
+        last_t = pe
         ev1.record(stream)
         torch.cuda.synchronize()
         barrier()
@@ -554,6 +603,15 @@ def run_ours(args):
     # bf16, the unfused launch pattern the pages contrast with one fused
     # launch.  Operands are gathered and scaled outside the timed region; it
     # runs last because it modifies W.
+    layerwise = None
+    if rank == 0 and world == 1 and not args.no_layerwise and not rebase and not topk:
+        layerwise = layerwise_graph(sw, cfg, routes, r_np, last_t if last_t is not None else 0,
+                                    stream)
+        if layerwise is not None:
+            layerwise["vs_single_launch"] = round(
+                statistics.mean(sw_real) / layerwise["ms"], 4)
+        assert sw.status(sh) == 0
+
     torch_base = None
     if rank == 0 and world == 1 and not args.no_torch_baseline and not rebase and T > 1:
         torch_base = torch_addmm_baseline(model, cfg, r_np, 0, 1, stream)
@@ -599,6 +657,7 @@ def run_ours(args):
                          "frac_of_this_gpu_copy": round(achieved / copy_gbs, 4)},
             "cpu_baseline": cpu,
             "torch_addmm_baseline": torch_base,
+            "layerwise_graph": layerwise,
             "e2e": e2e,
             "gpu_launches": 2 * args.steps,
             "router": router,
