@@ -46,7 +46,7 @@ def parse():
     ap.add_argument("--config", default="7b")
     ap.add_argument("--layers", type=int, default=None,
                     help="override the layer count (small cases for ncu captures)")
-    ap.add_argument("--kernel", choices=["auto", "mma", "tc", "tc2"], default="auto",
+    ap.add_argument("--kernel", choices=["auto", "mma", "tc", "tc2", "fold"], default="auto",
                     help="switch kernel: tensor-core (tc), tensor-core on CTA pairs (tc2), "
                          "mma.sync (mma), or auto")
     ap.add_argument("--mode", choices=["switch", "rebase"], default="switch",
@@ -60,6 +60,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-torch-baseline", action="store_true",
                     help="skip the unfused per-weight torch addmm_ context figure")
+    ap.add_argument("--schedule", choices=["dynamic", "static"], default="dynamic",
+                    help="tile schedule of the single-CTA tensor-core kernel")
     ap.add_argument("--no-layerwise", action="store_true",
                     help="skip the per-layer-launch CUDA graph context figure")
     return ap.parse_args()
@@ -72,6 +74,8 @@ KERNEL_SOURCES = {
     "switch_mma_kernel": ["common.cuh", "switch_mma.cuh"],
     "switch_tc2_kernel": ["common.cuh", "sm100_ptx.cuh", "switch_tc.cuh", "switch_tc2.cuh",
                           "switch_tc_host.cuh"],
+    "switch_fold_kernel": ["common.cuh", "sm100_ptx.cuh", "switch_tc.cuh", "switch_fold.cuh",
+                           "switch_tc_host.cuh"],
 }
 
 
@@ -437,10 +441,19 @@ def run_ours(args):
     sw = B.Switcher(model.W, model.A, model.B, cfg.n_layers, len(cfg.targets), cfg.n_experts,
                     cfg.rank, cfg.alpha, device=dev, names=[t.name for t in cfg.targets])
     sw.set_kernel({"auto": B.ADAFUSE_KERNEL_AUTO, "mma": B.ADAFUSE_KERNEL_MMA_SYNC,
-                   "tc": B.ADAFUSE_KERNEL_TCGEN05, "tc2": B.ADAFUSE_KERNEL_TCGEN05_PAIR}[args.kernel])
+                   "tc": B.ADAFUSE_KERNEL_TCGEN05, "tc2": B.ADAFUSE_KERNEL_TCGEN05_PAIR,
+                   "fold": B.ADAFUSE_KERNEL_TCGEN05_FOLD}[args.kernel])
+    sw.set_schedule(B.ADAFUSE_SCHEDULE_DYNAMIC if args.schedule == "dynamic"
+                    else B.ADAFUSE_SCHEDULE_STATIC)
+    # the kernel this run's switches launch (in-place top-k calls have their own choice)
+    kind = sw.topk_kernel if (args.top_k != 2 and args.mode != "rebase") else sw.kernel
     kernel_name = {B.ADAFUSE_KERNEL_MMA_SYNC: "switch_mma_kernel",
                    B.ADAFUSE_KERNEL_TCGEN05: "switch_tc_kernel",
-                   B.ADAFUSE_KERNEL_TCGEN05_PAIR: "switch_tc2_kernel"}[sw.kernel]
+                   B.ADAFUSE_KERNEL_TCGEN05_PAIR: "switch_tc2_kernel",
+                   B.ADAFUSE_KERNEL_TCGEN05_FOLD: "switch_fold_kernel"}[kind]
+    # the folded kernel's switch is two launches (fold, then switch); the
+    # events around a switch cover both
+    launches_per_switch = 2 if kind == B.ADAFUSE_KERNEL_TCGEN05_FOLD else 1
     rebase = args.mode == "rebase"
     if rebase:
         sw.set_base([w.clone() for w in model.W])
@@ -608,6 +621,7 @@ def run_ours(args):
         layerwise = layerwise_graph(sw, cfg, routes, r_np, last_t if last_t is not None else 0,
                                     stream)
         if layerwise is not None:
+            layerwise["launches_per_switch"] *= launches_per_switch
             layerwise["vs_single_launch"] = round(
                 statistics.mean(sw_real) / layerwise["ms"], 4)
         assert sw.status(sh) == 0
@@ -640,6 +654,7 @@ def run_ours(args):
                 "l2": "inputs larger than L2 (W read+write per switch >> 126 MB), no flush",
                 "parallelism": f"replicas x{world}",
                 "mode": args.mode,
+                "tile_schedule": args.schedule if kind == B.ADAFUSE_KERNEL_TCGEN05 else "static",
             },
             "switch_ms_p50": round(sw_sorted[len(sw_sorted) // 2], 4),
             "switch_ms_p90": round(sw_sorted[min(len(sw_sorted) - 1, int(0.9 * len(sw_sorted)))], 4),
@@ -659,7 +674,7 @@ def run_ours(args):
             "torch_addmm_baseline": torch_base,
             "layerwise_graph": layerwise,
             "e2e": e2e,
-            "gpu_launches": 2 * args.steps,
+            "gpu_launches": (1 + launches_per_switch) * args.steps,
             "router": router,
             "clocks": clocks,
         }

@@ -42,7 +42,8 @@
  * on it is in flight.  The library owns the context, its device-side
  * segment table and its device status word.  The library keeps no copy of W.
  * For ranks below 8 it keeps a zero-padded copy of every B (see
- * adafuse_refresh_adapters).
+ * adafuse_refresh_adapters); for ranks up to 8 a buffer the folded kernel
+ * rewrites from A on every switch (see ADAFUSE_KERNEL_TCGEN05_FOLD).
  *
  * Errors: every call returns ADAFUSE_OK (0) or a negative code.  Calls that
  * take a stream are asynchronous with respect to the host; host-side
@@ -90,6 +91,15 @@ extern "C" {
 #define ADAFUSE_KERNEL_TCGEN05   2  /* TMA + tcgen05/TMEM kernel, rank <= 8 or a multiple of 8 */
 #define ADAFUSE_KERNEL_TCGEN05_PAIR 3 /* the same on CTA pairs (tcgen05 cta_group::2, 256 x 128
                                          W blocks), rank a multiple of 8 */
+#define ADAFUSE_KERNEL_TCGEN05_FOLD 4 /* rank <= 8: the coefficients folded into the adapter
+                                         operand (c*A as three bf16 terms, written by a fold
+                                         launch before each switch launch), one TMEM
+                                         accumulator per tile; needs |c * A| within the
+                                         bf16 range */
+
+/* ---- tile schedules (adafuse_set_tile_schedule) ------------------------- */
+#define ADAFUSE_SCHEDULE_STATIC  0
+#define ADAFUSE_SCHEDULE_DYNAMIC 1
 
 /* One token's routing decision: the two chosen experts and their gates.
  * idx[j] == -1 marks an empty slot (its gate is ignored).  adafuse_pregate
@@ -191,12 +201,35 @@ ADAFUSE_API int adafuse_switch_batch_layers(adafuse_ctx* ctx, int32_t layer_begi
 /* Choose the kernel adafuse_switch launches for this context (default
  * ADAFUSE_KERNEL_AUTO).  All compute the same update to within the
  * documented rounding; ADAFUSE_KERNEL_TCGEN05 needs rank <= 8 or a multiple
- * of 8, ADAFUSE_KERNEL_TCGEN05_PAIR a multiple of 8 above 8; both return
- * UNSUPPORTED_SHAPE otherwise.  Host-only, no device work. */
+ * of 8, ADAFUSE_KERNEL_TCGEN05_PAIR a multiple of 8 above 8 and
+ * ADAFUSE_KERNEL_TCGEN05_FOLD rank <= 8; each returns UNSUPPORTED_SHAPE
+ * otherwise.  With ADAFUSE_KERNEL_TCGEN05_FOLD every switch, re-base or layer
+ * range is two launches on the stream: the fold of c_e * A_e for the route's
+ * experts into a context-owned buffer (at most 4 pairs of experts x 12 KB per
+ * 128 columns of every weight, allocated at create for ranks <= 8), then the
+ * switch.  Host-only, no device work. */
 ADAFUSE_API int adafuse_set_switch_kernel(adafuse_ctx* ctx, int kernel);
 
+/* The kernel adafuse_switch_topk and adafuse_switch_topk_layers launch: the
+ * context's choice, except that ADAFUSE_KERNEL_AUTO takes
+ * ADAFUSE_KERNEL_TCGEN05_FOLD for ranks <= 8 (an in-place top-k switch can
+ * touch 8 experts, which the folded kernel sums in one TMEM accumulator).
+ * Re-base calls follow adafuse_get_switch_kernel.  Host-only. */
+ADAFUSE_API int adafuse_get_topk_switch_kernel(adafuse_ctx* ctx);
+
+/* Tile schedule of ADAFUSE_KERNEL_TCGEN05 (the other kernels always use the
+ * static one).  ADAFUSE_SCHEDULE_STATIC: CTA b of the persistent grid takes
+ * tiles b, b + grid, b + 2*grid, ... of the segment table.
+ * ADAFUSE_SCHEDULE_DYNAMIC (default): each CTA takes its next tile from a
+ * context-owned ticket counter in table order, so the tiles in flight on the
+ * GPU stay a compact window of the table (neighbouring W rows) however far the
+ * CTAs' speeds drift apart; the launch leaves the counter at zero.
+ * INVALID_ARG for any other value.  Host-only, no device work. */
+ADAFUSE_API int adafuse_set_tile_schedule(adafuse_ctx* ctx, int schedule);
+
 /* The kernel adafuse_switch will launch (ADAFUSE_KERNEL_MMA_SYNC,
- * ADAFUSE_KERNEL_TCGEN05 or ADAFUSE_KERNEL_TCGEN05_PAIR), or a negative code. */
+ * ADAFUSE_KERNEL_TCGEN05, ADAFUSE_KERNEL_TCGEN05_PAIR or
+ * ADAFUSE_KERNEL_TCGEN05_FOLD), or a negative code. */
 ADAFUSE_API int adafuse_get_switch_kernel(adafuse_ctx* ctx);
 
 /* ---- re-base switch ------------------------------------------------------

@@ -18,10 +18,10 @@ from .util import (bf16_to_f64, bits, check_switch_rows, fp32_accum_gamma, make_
 
 pytestmark = pytest.mark.gpu
 
-MMA, TC, TC2 = (Bnd.ADAFUSE_KERNEL_MMA_SYNC, Bnd.ADAFUSE_KERNEL_TCGEN05,
-                Bnd.ADAFUSE_KERNEL_TCGEN05_PAIR)
+MMA, TC, TC2, TF = (Bnd.ADAFUSE_KERNEL_MMA_SYNC, Bnd.ADAFUSE_KERNEL_TCGEN05,
+                    Bnd.ADAFUSE_KERNEL_TCGEN05_PAIR, Bnd.ADAFUSE_KERNEL_TCGEN05_FOLD)
 # each kernel at a rank it takes
-KERNEL_RANKS = [(MMA, 8), (TC, 8), (TC, 4), (TC2, 16)]
+KERNEL_RANKS = [(MMA, 8), (TC, 8), (TC, 4), (TF, 8), (TF, 4), (TC2, 16)]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -183,7 +183,7 @@ def test_cuda_graph_capture_of_pregate_and_switch(kernel, r):
     assert torch.equal(r1[T - 1:T], cur)
 
 
-@pytest.mark.parametrize("kernel,r", [(TC, 8), (TC, 16), (TC2, 16), (TC2, 64)])
+@pytest.mark.parametrize("kernel,r", [(TC, 8), (TC, 16), (TF, 8), (TC2, 16), (TC2, 64)])
 def test_bounded_wait_timeout_reports_status_and_context_stays_usable(kernel, r):
     """Failure detection without a GPU fault: the test hook makes each CTA's
     first operand stage wait for 16 bytes that never arrive.  The MMA warp's
@@ -209,13 +209,13 @@ def test_stall_hook_is_refused_by_the_wait_free_kernel():
         Bnd.adafuse_debug_stall_next_switch(sw.ctx)
 
 
-@pytest.mark.parametrize("r", [1, 4, 7])
-def test_ranks_below_8_read_a_padded_copy_of_b_refreshed_on_request(r):
-    """Below rank 8 the tensor-core path reads B through the context's
+@pytest.mark.parametrize("kernel,r", [(TC, 1), (TC, 4), (TC, 7), (TF, 4)])
+def test_ranks_below_8_read_a_padded_copy_of_b_refreshed_on_request(kernel, r):
+    """Below rank 8 the tensor-core paths read B through the context's
     zero-padded copy.  After the caller changes B, adafuse_refresh_adapters
     brings the copy up to date and the switch matches the oracle on the new B."""
-    cfg, m, sw = _model(TC, seed=30 + r, r=r)
-    assert sw.kernel == TC
+    cfg, m, sw = _model(kernel, seed=30 + r, r=r)
+    assert sw.kernel == kernel
     routes = make_routes(np.array([[0, 2], [3, 1]], np.int32),
                          np.array([[0.7, 0.3], [0.6, 0.4]], np.float32))
     _switch_and_check(cfg, m, sw, routes, [(None, 0)])
@@ -224,3 +224,17 @@ def test_ranks_below_8_read_a_padded_copy_of_b_refreshed_on_request(r):
             b.mul_(-1.5)
     Bnd.adafuse_refresh_adapters(sw.ctx, stream())
     _switch_and_check(cfg, m, sw, routes, [(0, 1), (1, None)])
+
+
+@pytest.mark.parametrize("r", [8, 5])
+def test_folded_kernel_reads_a_afresh_on_every_switch(r):
+    """The folded kernel rebuilds c_e * A_e from A before every switch, so a
+    caller's in-place change of A needs no refresh call."""
+    cfg, m, sw = _model(TF, seed=40 + r, r=r)
+    routes = make_routes(np.array([[0, 2], [3, 1], [1, 2]], np.int32),
+                         np.array([[0.7, 0.3], [0.6, 0.4], [0.5, 0.5]], np.float32))
+    _switch_and_check(cfg, m, sw, routes, [(None, 0), (0, 1)])
+    with torch.no_grad():
+        for a in m.A:
+            a.mul_(-0.75)
+    _switch_and_check(cfg, m, sw, routes, [(1, 2), (2, None)])

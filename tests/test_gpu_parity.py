@@ -38,8 +38,8 @@ def stream():
     return torch.cuda.current_stream().cuda_stream
 
 
-MMA, TC, TC2 = (Bnd.ADAFUSE_KERNEL_MMA_SYNC, Bnd.ADAFUSE_KERNEL_TCGEN05,
-                Bnd.ADAFUSE_KERNEL_TCGEN05_PAIR)
+MMA, TC, TC2, TF = (Bnd.ADAFUSE_KERNEL_MMA_SYNC, Bnd.ADAFUSE_KERNEL_TCGEN05,
+                    Bnd.ADAFUSE_KERNEL_TCGEN05_PAIR, Bnd.ADAFUSE_KERNEL_TCGEN05_FOLD)
 
 
 def make_switcher(model: wl.Model, kernel: int = Bnd.ADAFUSE_KERNEL_AUTO) -> Bnd.Switcher:
@@ -55,12 +55,12 @@ def make_switcher(model: wl.Model, kernel: int = Bnd.ADAFUSE_KERNEL_AUTO) -> Bnd
 
 def kernels_for(rank):
     if rank <= 8:
-        return [MMA, TC]
+        return [MMA, TC, TF]
     return [MMA, TC, TC2] if rank % 8 == 0 else [MMA]
 
 
 # (kernel, rank) for the small-model tests: each kernel at a rank it takes
-KERNEL_RANKS = [(MMA, 8), (TC, 8), (TC2, 16)]
+KERNEL_RANKS = [(MMA, 8), (TC, 8), (TF, 8), (TF, 3), (TC2, 16)]
 
 
 def host_ab(model):
@@ -278,6 +278,33 @@ def test_layer_ranges_equal_one_full_switch(kernel, r):
         s2.switch_layers(2, 2, p(0), p(1), stream())
 
 
+@pytest.mark.parametrize("r", [8, 4, 16])
+def test_static_and_dynamic_tile_schedules_agree_bitwise(r):
+    """The schedule only decides which CTA takes a tile, never how a tile is
+    computed: a static and a dynamic context give the same W, bit for bit,
+    over repeated full and layer-range launches (the dynamic ticket counter
+    is back at zero after every launch)."""
+    m1, m2 = _small_model(seed=12, r=r), _small_model(seed=12, r=r)
+    s1, s2 = make_switcher(m1, TC), make_switcher(m2, TC)
+    s1.set_schedule(Bnd.ADAFUSE_SCHEDULE_STATIC)
+    s2.set_schedule(Bnd.ADAFUSE_SCHEDULE_DYNAMIC)
+    routes = make_routes(np.array([[0, 1], [2, 3], [1, 2], [3, 0]], np.int32),
+                         np.array([[0.7, 0.3], [0.6, 0.4], [0.5, 0.5], [0.9, 0.1]], np.float32))
+    p = lambda t: Bnd.Switcher.route_ptr(routes, t)
+    for sw in (s1, s2):
+        sw.switch(None, p(0), stream())
+        sw.switch(p(0), p(1), stream())
+        sw.switch_layers(1, 1, p(1), p(2), stream())
+        sw.switch_layers(0, 1, p(1), p(2), stream())
+        sw.switch(p(2), p(3), stream())
+    torch.cuda.synchronize()
+    assert s1.status(stream()) == 0 and s2.status(stream()) == 0
+    for a, b in zip(m1.W, m2.W):
+        assert torch.equal(a, b)
+    with pytest.raises(Bnd.AdafuseError):
+        s1.set_schedule(7)
+
+
 @pytest.mark.parametrize("kernel,r", KERNEL_RANKS)
 @pytest.mark.parametrize("bad", ["index_high", "index_low", "gate_nan", "gate_inf"])
 def test_bad_route_sets_status_and_writes_nothing(bad, kernel, r):
@@ -339,7 +366,7 @@ def _full_size_case(name, n_switches, full_first=True, kernel=Bnd.ADAFUSE_KERNEL
     torch.cuda.empty_cache()
     model = wl.make_model(cfg, device="cuda")
     sw = make_switcher(model, kernel)
-    assert sw.kernel in (TC, TC2)  # a tensor-core kernel, as the benchmark launches
+    assert sw.kernel in (TC, TC2, TF)  # a tensor-core kernel, as the benchmark launches
     A_h, B_h = host_ab(model)
     if cfg.route_mode == "router":
         h = wl.make_hidden(cfg, T=n_switches, device="cuda")
@@ -365,16 +392,23 @@ def test_auto_picks_tensor_cores_when_rank_allows():
         cfg = wl.custom("k", 1, [("q", 64, 64)], n_experts=2, rank=r, alpha=2.0 * r, n_tokens=1)
         sw = make_switcher(wl.make_model(cfg, device="cuda"))
         assert sw.kernel == want
+        # in-place top-k switches take the folded kernel wherever it runs
+        assert sw.topk_kernel == (TF if r <= 8 else want)
         if want == MMA:
             with pytest.raises(Bnd.AdafuseError):
                 sw.set_kernel(TC)
         if r <= 8:
             with pytest.raises(Bnd.AdafuseError):
                 sw.set_kernel(TC2)
+            sw.set_kernel(TF)
+        else:
+            with pytest.raises(Bnd.AdafuseError):
+                sw.set_kernel(TF)
 
 
-def test_llama2_7b_shape_sampled():
-    _full_size_case("7b", 3)
+@pytest.mark.parametrize("kernel", [Bnd.ADAFUSE_KERNEL_AUTO, TC, TF])
+def test_llama2_7b_shape_sampled(kernel):
+    _full_size_case("7b", 3, kernel=kernel)
 
 
 @pytest.mark.parametrize("kernel", [Bnd.ADAFUSE_KERNEL_AUTO, TC, TC2])

@@ -18,8 +18,8 @@ from .util import bits, check_switch_rows, make_routes, route_tuple, routes_to_n
 
 pytestmark = pytest.mark.gpu
 
-MMA, TC, TC2 = (Bnd.ADAFUSE_KERNEL_MMA_SYNC, Bnd.ADAFUSE_KERNEL_TCGEN05,
-                Bnd.ADAFUSE_KERNEL_TCGEN05_PAIR)
+MMA, TC, TC2, TF = (Bnd.ADAFUSE_KERNEL_MMA_SYNC, Bnd.ADAFUSE_KERNEL_TCGEN05,
+                    Bnd.ADAFUSE_KERNEL_TCGEN05_PAIR, Bnd.ADAFUSE_KERNEL_TCGEN05_FOLD)
 SHAPES = [("a", 200, 136), ("b", 264, 392), ("c", 128, 256), ("d", 8, 8)]
 
 
@@ -59,7 +59,7 @@ def _check_against_oracle(cfg, m, W0, route, A_h, B_h):
 @pytest.mark.parametrize("E,r,kernel", [(3, 3, MMA), (4, 8, MMA), (4, 8, TC), (5, 16, TC),
                                         (3, 24, MMA), (4, 32, TC), (6, 64, TC), (5, 16, TC2),
                                         (3, 24, TC2), (4, 32, TC2), (6, 64, TC2), (3, 3, TC),
-                                        (4, 4, TC)])
+                                        (4, 4, TC), (4, 8, TF), (3, 3, TF)])
 def test_rebase_matches_oracle_and_does_not_accumulate(E, r, kernel):
     cfg, m, sw, W0 = _setup(E, r, kernel, seed=31 * r + E)
     W0_bits = [bits(w) for w in W0]
@@ -84,7 +84,7 @@ def test_rebase_matches_oracle_and_does_not_accumulate(E, r, kernel):
         assert np.array_equal(bits(w0), b0)
 
 
-@pytest.mark.parametrize("kernel,r", [(MMA, 8), (TC, 8), (TC2, 16)])
+@pytest.mark.parametrize("kernel,r", [(MMA, 8), (TC, 8), (TF, 8), (TC2, 16)])
 def test_rebase_layer_ranges_equal_full(kernel, r):
     cfg, m1, s1, _ = _setup(4, r, kernel, seed=3, layers=3)
     _, m2, s2, _ = _setup(4, r, kernel, seed=3, layers=3)
@@ -98,7 +98,7 @@ def test_rebase_layer_ranges_equal_full(kernel, r):
         assert torch.equal(a, b)
 
 
-@pytest.mark.parametrize("kernel,r", [(MMA, 8), (TC, 8), (TC2, 16)])
+@pytest.mark.parametrize("kernel,r", [(MMA, 8), (TC, 8), (TF, 8), (TC2, 16)])
 def test_rebase_bad_route_writes_nothing(kernel, r):
     cfg, m, sw, _ = _setup(4, r, kernel, seed=4)
     before = [bits(w) for w in m.W]

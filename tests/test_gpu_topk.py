@@ -21,8 +21,8 @@ from .util import (bits, check_switch_rows, make_routes4, pregate_topk_consisten
 
 pytestmark = pytest.mark.gpu
 
-MMA, TC, TC2 = (Bnd.ADAFUSE_KERNEL_MMA_SYNC, Bnd.ADAFUSE_KERNEL_TCGEN05,
-                Bnd.ADAFUSE_KERNEL_TCGEN05_PAIR)
+MMA, TC, TC2, TF = (Bnd.ADAFUSE_KERNEL_MMA_SYNC, Bnd.ADAFUSE_KERNEL_TCGEN05,
+                    Bnd.ADAFUSE_KERNEL_TCGEN05_PAIR, Bnd.ADAFUSE_KERNEL_TCGEN05_FOLD)
 GATE_RTOL = 1e-5
 
 
@@ -48,7 +48,7 @@ def switcher(model, kernel=Bnd.ADAFUSE_KERNEL_AUTO):
 
 def kernels_for(rank):
     if rank <= 8:
-        return [MMA, TC]
+        return [MMA, TC, TF]
     return [MMA, TC, TC2] if rank % 8 == 0 else [MMA]
 
 
@@ -198,7 +198,7 @@ def _small(seed=3, E=8, r=16):
     return wl.make_model(cfg, device="cuda", seed=seed)
 
 
-KERNEL_RANKS = [(MMA, 8), (TC, 8), (TC, 4), (TC, 16), (TC2, 16)]
+KERNEL_RANKS = [(MMA, 8), (TC, 8), (TC, 4), (TF, 8), (TF, 4), (TC, 16), (TC2, 16)]
 
 
 @pytest.mark.parametrize("kernel,r", KERNEL_RANKS)

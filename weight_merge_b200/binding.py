@@ -28,6 +28,9 @@ ADAFUSE_KERNEL_AUTO = 0
 ADAFUSE_KERNEL_MMA_SYNC = 1
 ADAFUSE_KERNEL_TCGEN05 = 2
 ADAFUSE_KERNEL_TCGEN05_PAIR = 3
+ADAFUSE_KERNEL_TCGEN05_FOLD = 4
+ADAFUSE_SCHEDULE_STATIC = 0
+ADAFUSE_SCHEDULE_DYNAMIC = 1
 ADAFUSE_MAX_TOP_K = 4
 
 
@@ -86,6 +89,8 @@ def lib() -> ctypes.CDLL:
         "adafuse_switch_batch_layers": ([P, i32, i32, P, P, P], ctypes.c_int),
         "adafuse_get_device_status": ([P, P, ctypes.POINTER(i32)], ctypes.c_int),
         "adafuse_set_switch_kernel": ([P, ctypes.c_int], ctypes.c_int),
+        "adafuse_set_tile_schedule": ([P, ctypes.c_int], ctypes.c_int),
+        "adafuse_get_topk_switch_kernel": ([P], ctypes.c_int),
         "adafuse_set_base": ([P, ctypes.POINTER(P)], ctypes.c_int),
         "adafuse_rebase": ([P, P, P], ctypes.c_int),
         "adafuse_rebase_layers": ([P, i32, i32, P, P], ctypes.c_int),
@@ -202,6 +207,17 @@ def adafuse_debug_stall_next_switch(ctx: int) -> None:
 
 def adafuse_set_switch_kernel(ctx: int, kernel: int) -> None:
     _check(lib().adafuse_set_switch_kernel(ctx, int(kernel)), "adafuse_set_switch_kernel")
+
+
+def adafuse_set_tile_schedule(ctx: int, schedule: int) -> None:
+    _check(lib().adafuse_set_tile_schedule(ctx, int(schedule)), "adafuse_set_tile_schedule")
+
+
+def adafuse_get_topk_switch_kernel(ctx: int) -> int:
+    k = lib().adafuse_get_topk_switch_kernel(ctx)
+    if k < 0:
+        _check(k, "adafuse_get_topk_switch_kernel")
+    return k
 
 
 def adafuse_get_switch_kernel(ctx: int) -> int:
@@ -325,9 +341,16 @@ class Switcher:
     def set_kernel(self, kernel: int) -> None:
         adafuse_set_switch_kernel(self.ctx, kernel)
 
+    def set_schedule(self, schedule: int) -> None:
+        adafuse_set_tile_schedule(self.ctx, schedule)
+
     @property
     def kernel(self) -> int:
         return adafuse_get_switch_kernel(self.ctx)
+
+    @property
+    def topk_kernel(self) -> int:
+        return adafuse_get_topk_switch_kernel(self.ctx)
 
     def status(self, stream: int = 0) -> int:
         return adafuse_get_device_status(self.ctx, stream)

@@ -40,6 +40,9 @@ struct adafuse_ctx {
     // pair kernel: 256 x 128 blocks, layer-major like the tile table
     TileEntry* d_blocks = nullptr;
     uint16_t* d_bpad = nullptr;              // rank < 8: B with rows zero-padded to 8
+    uint16_t* d_fold = nullptr;              // rank <= 8: folded-coefficient operands
+    unsigned long long* d_sched = nullptr;   // [2] ticket counter of the dynamic tile schedule
+    int schedule = ADAFUSE_SCHEDULE_DYNAMIC;
     std::vector<int64_t> layer_block_begin;  // [n_layers + 1]
     int pair_clusters = 0;                   // co-resident CTA pairs (0 = not queried yet)
 };
@@ -130,6 +133,9 @@ int64_t walk_blocks(const adafuse_desc* d, Emit&& emit) {
 // tensor maps fetch exactly 8 rows for the single-CTA kernel's layout).
 bool pair_eligible(const adafuse_ctx* c) { return c->tc_kp != 0 && c->rank > 8; }
 
+// The folded kernel takes ranks up to 8 once its operand buffer exists.
+bool fold_eligible(const adafuse_ctx* c) { return c->tc_kp != 0 && c->d_fold != nullptr; }
+
 // Rank < 8: copy every B [E, out, r] into its [E, out, 8] zero-padded slot
 // (the padding columns are zeroed once, at create).
 cudaError_t copy_padded_b(const adafuse_ctx* c, cudaStream_t s) {
@@ -164,6 +170,8 @@ cudaError_t launch_tc(adafuse_ctx* c, int64_t t0, int64_t t1, const int32_t* pre
     prm.w0_maps = c->d_w0_maps;
     prm.stall = c->stall_next ? 1 : 0;
     c->stall_next = false;
+    prm.dyn = c->schedule == ADAFUSE_SCHEDULE_DYNAMIC ? 1 : 0;
+    prm.sched = c->d_sched;
     return launch_switch_tc<KP, BBULK>(prm, c->device, c->sm_count, s);
 }
 
@@ -193,6 +201,8 @@ cudaError_t launch_tc2(adafuse_ctx* c, int64_t b0, int64_t b1, const int32_t* pr
     prm.w0_maps = c->d_w0_maps;
     prm.stall = c->stall_next ? 1 : 0;
     c->stall_next = false;
+    prm.dyn = 0;
+    prm.sched = nullptr;
     return launch_switch_tc2<KP>(prm, c->pair_clusters, s);
 }
 
@@ -272,6 +282,7 @@ int adafuse_create(adafuse_ctx** out, const adafuse_desc* desc, int device) {
         pairs[i].A = static_cast<const uint16_t*>(t.A);
         pairs[i].B = static_cast<const uint16_t*>(t.B);
         pairs[i].Bk = pairs[i].B;
+        pairs[i].Af = nullptr;
         pairs[i].out = (int32_t)t.out;
         pairs[i].in = (int32_t)t.in;
         pairs[i].layer = (int32_t)(i / desc->n_targets);
@@ -309,6 +320,8 @@ int adafuse_create(adafuse_ctx** out, const adafuse_desc* desc, int device) {
         cudaFree(c->d_maps);
         cudaFree(c->d_blocks);
         cudaFree(c->d_bpad);
+        cudaFree(c->d_fold);
+        cudaFree(c->d_sched);
         delete c;
         return err == cudaErrorMemoryAllocation ? ADAFUSE_ERR_OUT_OF_MEMORY : cuda_fail(err, what);
     };
@@ -330,12 +343,30 @@ int adafuse_create(adafuse_ctx** out, const adafuse_desc* desc, int device) {
         if ((e = copy_padded_b(c, nullptr)) != cudaSuccess) return fail(e, "cudaMemcpy2D(padded B)");
         if ((e = cudaDeviceSynchronize()) != cudaSuccess) return fail(e, "padded B");
     }
+    // ranks up to 8: room for the folded operand of up to four expert pairs
+    // per 128-column block of every weight (written by each folded switch)
+    if (desc->rank <= 8 && tc_kp_for(desc->rank) != 0) {
+        size_t total = 0;
+        for (const PairDesc& pd : pairs) total += fold_bytes_for(pd.in);
+        if ((e = cudaMalloc(&c->d_fold, total)) != cudaSuccess)
+            return fail(e, "cudaMalloc(folded operands)");
+        size_t off = 0;
+        for (PairDesc& pd : pairs) {
+            pd.Af = c->d_fold + off / 2;
+            off += fold_bytes_for(pd.in);
+        }
+        c->h_pairs = pairs;
+    }
     if ((e = cudaMalloc(&c->d_pairs, sizeof(PairDesc) * pairs.size())) != cudaSuccess)
         return fail(e, "cudaMalloc(pairs)");
     if ((e = cudaMalloc(&c->d_tiles, sizeof(TileEntry) * tiles.size())) != cudaSuccess)
         return fail(e, "cudaMalloc(tiles)");
     if ((e = cudaMalloc(&c->d_status, sizeof(int32_t))) != cudaSuccess)
         return fail(e, "cudaMalloc(status)");
+    if ((e = cudaMalloc(&c->d_sched, 2 * sizeof(unsigned long long))) != cudaSuccess)
+        return fail(e, "cudaMalloc(schedule)");
+    if ((e = cudaMemset(c->d_sched, 0, 2 * sizeof(unsigned long long))) != cudaSuccess)
+        return fail(e, "cudaMemset(schedule)");
     if ((e = cudaMemcpy(c->d_pairs, pairs.data(), sizeof(PairDesc) * pairs.size(),
                         cudaMemcpyHostToDevice)) != cudaSuccess)
         return fail(e, "cudaMemcpy(pairs)");
@@ -408,6 +439,8 @@ int adafuse_destroy(adafuse_ctx* ctx) {
     cudaFree(ctx->d_w0_maps);
     cudaFree(ctx->d_blocks);
     cudaFree(ctx->d_bpad);
+    cudaFree(ctx->d_fold);
+    cudaFree(ctx->d_sched);
     delete ctx;
     return ADAFUSE_OK;
 }
@@ -415,12 +448,32 @@ int adafuse_destroy(adafuse_ctx* ctx) {
 int adafuse_set_switch_kernel(adafuse_ctx* ctx, int kernel) {
     if (ctx == nullptr) return ADAFUSE_ERR_INVALID_ARG;
     if (kernel != ADAFUSE_KERNEL_AUTO && kernel != ADAFUSE_KERNEL_MMA_SYNC &&
-        kernel != ADAFUSE_KERNEL_TCGEN05 && kernel != ADAFUSE_KERNEL_TCGEN05_PAIR)
+        kernel != ADAFUSE_KERNEL_TCGEN05 && kernel != ADAFUSE_KERNEL_TCGEN05_PAIR &&
+        kernel != ADAFUSE_KERNEL_TCGEN05_FOLD)
         return ADAFUSE_ERR_INVALID_ARG;
     if (kernel == ADAFUSE_KERNEL_TCGEN05 && ctx->tc_kp == 0) return ADAFUSE_ERR_UNSUPPORTED_SHAPE;
     if (kernel == ADAFUSE_KERNEL_TCGEN05_PAIR && !pair_eligible(ctx))
         return ADAFUSE_ERR_UNSUPPORTED_SHAPE;
+    if (kernel == ADAFUSE_KERNEL_TCGEN05_FOLD && !fold_eligible(ctx))
+        return ADAFUSE_ERR_UNSUPPORTED_SHAPE;
     ctx->kernel = kernel;
+    return ADAFUSE_OK;
+}
+
+int adafuse_get_topk_switch_kernel(adafuse_ctx* ctx) {
+    if (ctx == nullptr) return ADAFUSE_ERR_INVALID_ARG;
+    // measured on B200 at the Llama-2-7B shape, top-4 in place: the folded
+    // kernel's single accumulator holds up to 8 experts (79% of peak), where
+    // the four-accumulator kernel needs two TMEM passes per tile (58%)
+    if (ctx->kernel == ADAFUSE_KERNEL_AUTO && fold_eligible(ctx)) return ADAFUSE_KERNEL_TCGEN05_FOLD;
+    return adafuse_get_switch_kernel(ctx);
+}
+
+int adafuse_set_tile_schedule(adafuse_ctx* ctx, int schedule) {
+    if (ctx == nullptr) return ADAFUSE_ERR_INVALID_ARG;
+    if (schedule != ADAFUSE_SCHEDULE_STATIC && schedule != ADAFUSE_SCHEDULE_DYNAMIC)
+        return ADAFUSE_ERR_INVALID_ARG;
+    ctx->schedule = schedule;
     return ADAFUSE_OK;
 }
 
@@ -528,7 +581,8 @@ int launch_switch(adafuse_ctx* ctx, int32_t layer_begin, int32_t n_layers,
     DeviceGuard guard(ctx->device);
     if (!guard.ok) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const int kind = adafuse_get_switch_kernel(ctx);
+    const int kind = slots == 4 && !rebase ? adafuse_get_topk_switch_kernel(ctx)
+                                           : adafuse_get_switch_kernel(ctx);
     if (kind == ADAFUSE_KERNEL_TCGEN05_PAIR) {
         const int64_t b0 = ctx->layer_block_begin[(size_t)layer_begin];
         const int64_t b1 = ctx->layer_block_begin[(size_t)layer_begin + n_layers];
@@ -539,6 +593,31 @@ int launch_switch(adafuse_ctx* ctx, int32_t layer_begin, int32_t n_layers,
             e = launch_tc2<32>(ctx, b0, b1, prev, cur, slots, s, rebase);
         else
             e = launch_tc2<64>(ctx, b0, b1, prev, cur, slots, s, rebase);
+        return e == cudaSuccess ? ADAFUSE_OK : cuda_fail(e, "switch launch");
+    }
+    if (kind == ADAFUSE_KERNEL_TCGEN05_FOLD) {
+        TcParams prm;
+        prm.pairs = ctx->d_pairs;
+        prm.tiles = ctx->d_tiles;
+        prm.maps = ctx->d_maps;
+        prm.t_begin = t0;
+        prm.t_end = t1;
+        prm.prev = prev;
+        prm.cur = cur;
+        prm.slots = slots;
+        prm.E = ctx->n_experts;
+        prm.s = ctx->scale;
+        prm.status = ctx->d_status;
+        prm.rebase = rebase ? 1 : 0;
+        prm.w0_maps = ctx->d_w0_maps;
+        prm.stall = ctx->stall_next ? 1 : 0;
+        ctx->stall_next = false;
+        prm.dyn = 0;
+        prm.sched = nullptr;
+        const int64_t w0 = (int64_t)layer_begin * ctx->n_targets;
+        const int64_t nw = (int64_t)n_layers * ctx->n_targets;
+        const cudaError_t e =
+            launch_switch_fold(prm, w0, nw, ctx->rank, ctx->device, ctx->sm_count, s);
         return e == cudaSuccess ? ADAFUSE_OK : cuda_fail(e, "switch launch");
     }
     if (kind == ADAFUSE_KERNEL_TCGEN05) {

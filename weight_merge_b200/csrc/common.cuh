@@ -20,6 +20,8 @@ struct PairDesc {
     const uint16_t* W0;  // [out, in] pristine base for the re-base switch (or null)
     const uint16_t* Bk;  // [E, out, 8] B with 16-byte rows for the rank <= 8 tensor-core
                          // path: B itself at rank 8, a zero-padded copy below
+    uint16_t* Af;        // rank <= 8: the folded-coefficient operand the fold launch
+                         // writes before each folded switch (or null)
     int32_t out;
     int32_t in;
     int32_t layer;

@@ -69,8 +69,10 @@ struct TcConfig {
                                        : KP == 32 ? sm100::kSwizzle64B
                                                   : sm100::kSwizzle128B;
     static constexpr uint32_t kBSbo = 8 * KP * 2;          // 8 rows of the swizzled B slice
-    // barriers + tmem base + abort flag, after the data
-    static constexpr uint32_t kBarBytes = 8 * (3 * kWStages + 2 * kOpStages + 2) + 16;
+    // barriers (w_full, w_empty, epi_done, te_full per W stage; op_full,
+    // op_empty per operand stage; acc_full, acc_empty), the W stages' tile
+    // entries, tmem base + abort flag, after the data
+    static constexpr uint32_t kBarBytes = 8 * (4 * kWStages + 2 * kOpStages + 2) + 8 * kWStages + 16;
     static constexpr uint32_t kSmemBytes =
         1024 /*alignment slack*/ + kOpBytes + kZeroBytes + kWBytes + kBarBytes;
     static_assert(kSmemBytes <= 232448, "shared memory");
@@ -97,7 +99,16 @@ struct TcParams {
     // than its loads deliver, so the MMA warp's bounded wait runs out and the
     // launch ends through the timeout path before any MMA completes
     int stall;
+    // tile schedule: 0 = static (CTA b takes tiles b, b + grid, ...); 1 =
+    // dynamic (the W producers take tickets from sched[0] in table order, so
+    // the tiles in flight stay a compact window of the table however the
+    // CTAs' speeds drift apart; the last CTA to finish zeroes sched[0..1])
+    int dyn;
+    unsigned long long* sched;
 };
+
+// End-of-schedule marker in a W stage's tile-entry slot.
+constexpr uint32_t kTileEndX = 0xffffffffu;
 
 // Tile entries are fetched one iteration ahead (the loops below keep the next
 // entry in a register), so no tile waits on a dependent global load.
@@ -189,7 +200,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
     uint64_t* acc_full = op_empty + C::kOpStages;
     uint64_t* acc_empty = acc_full + 1;
     uint64_t* epi_done = acc_empty + 1;            // [kWStages]: epilogue wrote the tile
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epi_done + C::kWStages);
+    uint64_t* te_full = epi_done + C::kWStages;    // [kWStages]: the stage's tile entry is set
+    TileEntry* te_slot = reinterpret_cast<TileEntry*>(te_full + C::kWStages);  // [kWStages]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(te_slot + C::kWStages);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     Coefs8 cf;
@@ -200,7 +213,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
     }
     if (cf.n == 0 && !p.rebase) return;  // identity switch
     const int64_t first = p.t_begin + blockIdx.x;
-    if (first >= p.t_end) return;
+    // (the dynamic schedule needs every CTA at teardown to reset its counter;
+    // the launch never has more CTAs than tiles, so no CTA leaves here then)
+    if (!p.dyn && first >= p.t_end) return;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -215,6 +230,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
             mbar_init(&w_full[i], 1);
             mbar_init(&w_empty[i], 1);
             mbar_init(&epi_done[i], kTcEpiThreads);
+            mbar_init(&te_full[i], 1);
         }
         for (int i = 0; i < C::kOpStages; ++i) {
             mbar_init(&op_full[i], 1);
@@ -244,43 +260,68 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
 
     if (warp == 0) {
         // ---------------- W producer: tiles into the W ring ----
-        // Runs ahead of everything else, limited only by free W stages.
+        // Runs ahead of everything else, limited only by free W stages.  It
+        // picks the tiles (the next ticket is taken one tile ahead) and
+        // publishes each stage's tile entry, or the end marker, to the other
+        // roles through te_slot / te_full.
         if (lane == 0) {
             int ws = 0;
             uint32_t wph = 0;
             uint32_t last_pair = 0xffffffffu;
-            TileEntry te_next = fetch_tile(p.tiles, first, p.t_end);
-            for (int64_t t = first; t < p.t_end && !*abort_flag; t += gridDim.x) {
-                const TileInfo ti = decode_tile(te_next);
-                te_next = fetch_tile(p.tiles, t + gridDim.x, p.t_end);
+            auto next_tile = [&](int64_t t) -> int64_t {
+                if (t >= p.t_end) return t;
+                return p.dyn ? p.t_begin + (int64_t)atomicAdd(p.sched, 1ull) : t + gridDim.x;
+            };
+            int64_t t = p.dyn ? next_tile(p.t_begin) : first;
+            TileEntry te = fetch_tile(p.tiles, t, p.t_end);
+            while (!*abort_flag) {
+                const int64_t tn = next_tile(t);
+                const TileEntry te_n = fetch_tile(p.tiles, tn, p.t_end);
+                if (!mbar_wait_bounded(&w_empty[ws], wph ^ 1, abort_flag, kWaitLimitNs)) { fail(1); break; }
+                if (t >= p.t_end) {
+                    te_slot[ws] = make_uint2(kTileEndX, kTileEndX);
+                    mbar_arrive(&te_full[ws]);
+                    break;
+                }
+                te_slot[ws] = te;
+                mbar_arrive(&te_full[ws]);
+                const TileInfo ti = decode_tile(te);
                 const CUtensorMap* mW = p.rebase ? p.w0_maps + ti.pair : p.maps + 3 * (size_t)ti.pair;
                 if (ti.pair != last_pair) {
                     tensormap_acquire(mW);
                     last_pair = ti.pair;
                 }
-                if (!mbar_wait_bounded(&w_empty[ws], wph ^ 1, abort_flag, kWaitLimitNs)) { fail(1); break; }
                 uint8_t* wdst = w_ring + (size_t)ws * kWTileBytes;
                 mbar_arrive_expect_tx(&w_full[ws], ti.wide ? kWTileBytes : kWBoxBytes);
                 tma_load_2d(wdst, mW, ti.col0, ti.row0, &w_full[ws]);
                 if (ti.wide) tma_load_2d(wdst + kWBoxBytes, mW, ti.col0 + 64, ti.row0, &w_full[ws]);
                 if (++ws == C::kWStages) { ws = 0; wph ^= 1; }
-                if (t + gridDim.x < p.t_end && (te_next.x & kTilePairMask) != ti.pair) {
-                    const uint32_t np = te_next.x & kTilePairMask;
+                if (tn < p.t_end && (te_n.x & kTilePairMask) != ti.pair) {
+                    const uint32_t np = te_n.x & kTilePairMask;
                     tensormap_prefetch(p.rebase ? p.w0_maps + np : p.maps + 3 * (size_t)np);
+                    tensormap_prefetch(p.maps + 3 * (size_t)np + 1);
+                    tensormap_prefetch(p.maps + 3 * (size_t)np + 2);
                 }
+                t = tn;
+                te = te_n;
             }
         }
     } else if (warp == 3) {
         // ---------------- operand producer: per tile and expert, the B-row and
         // A-column slices into the operand ring (paced by the MMA warp) ----
         if (lane == 0) {
-            int os = 0;
-            uint32_t oph = 0;
+            int os = 0, ts = 0;
+            uint32_t oph = 0, tph = 0;
             uint32_t last_pair = 0xffffffffu;
-            TileEntry te_next = fetch_tile(p.tiles, first, p.t_end);
-            for (int64_t t = first; t < p.t_end && !*abort_flag; t += gridDim.x) {
-                const TileInfo ti = decode_tile(te_next);
-                te_next = fetch_tile(p.tiles, t + gridDim.x, p.t_end);
+            bool first_tile = true;
+            while (!*abort_flag) {
+                if (!mbar_wait_bounded(&te_full[ts], tph, abort_flag, kWaitLimitNs)) { fail(8); break; }
+                const TileEntry te = te_slot[ts];
+                if (++ts == C::kWStages) { ts = 0; tph ^= 1; }
+                if (te.x == kTileEndX) break;
+                const bool stall_here = p.stall && first_tile;
+                first_tile = false;
+                const TileInfo ti = decode_tile(te);
                 const uint32_t pair = ti.pair;
                 const int row0 = ti.row0, col0 = ti.col0;
                 const CUtensorMap* mA = p.maps + 3 * (size_t)pair + 1;
@@ -312,11 +353,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
                         // products only reach accumulator rows never stored)
                         const uint32_t bbytes = (uint32_t)out_rows * 16u;
                         mbar_arrive_expect_tx(&op_full[os], bbytes + (second ? 2 : 1) * C::kAHalfBytes +
-                                                                (p.stall && t == first && ei == 0 ? kStallBytes : 0u));
+                                                                (stall_here && ei == 0 ? kStallBytes : 0u));
                         bulk_load(b_dst, Bbase + ((size_t)e * out + row0) * 8, bbytes, &op_full[os]);
                     } else {
                         mbar_arrive_expect_tx(&op_full[os], C::kBBytes + (second ? 2 : 1) * C::kAHalfBytes +
-                                                                (p.stall && t == first && ei == 0 ? kStallBytes : 0u));
+                                                                (stall_here && ei == 0 ? kStallBytes : 0u));
                         tma_load_3d(b_dst, mB, 0, row0, e, &op_full[os]);
                     }
                     tma_load_3d(a_dst, mA, col0, 0, e, &op_full[os]);
@@ -324,11 +365,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
                     if (++os == C::kOpStages) { os = 0; oph ^= 1; }
                 }
                 if (!ok) { fail(2); break; }
-                if (t + gridDim.x < p.t_end && (te_next.x & kTilePairMask) != pair) {
-                    const CUtensorMap* nm = p.maps + 3 * (size_t)(te_next.x & kTilePairMask);
-                    tensormap_prefetch(nm + 1);
-                    tensormap_prefetch(nm + 2);
-                }
             }
         }
     } else if (warp == 1) {
@@ -336,11 +372,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
         if (lane == 0) {
             constexpr uint32_t idesc = instr_desc_bf16(128, 128, /*B MN-major*/ 1);
             const uint32_t zero_s = smem_u32(zero_blk);
-            int os = 0;
-            uint32_t oph = 0, aph = 0;
+            int os = 0, ts = 0;
+            uint32_t oph = 0, aph = 0, tph = 0;
             const int nb = tmem_batches(cf);
             bool ok = true;
-            for (int64_t t = first; t < p.t_end && ok && !*abort_flag; t += gridDim.x) {
+            while (ok && !*abort_flag) {
+                if (!mbar_wait_bounded(&te_full[ts], tph, abort_flag, kWaitLimitNs)) { fail(9); break; }
+                const bool end = te_slot[ts].x == kTileEndX;
+                if (++ts == C::kWStages) { ts = 0; tph ^= 1; }
+                if (end) break;
 #pragma unroll 1
               for (int b0 = 0; b0 < nb * kTmemBatch && ok; b0 += kTmemBatch) {
                 if (!mbar_wait_bounded(acc_empty, aph ^ 1, abort_flag, kWaitLimitNs)) { fail(3); ok = false; break; }
@@ -391,10 +431,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
             if (lane == 0) {
                 int ws = 0;
                 uint32_t wph = 0;
-                TileEntry te_next = fetch_tile(p.tiles, first, p.t_end);
-                for (int64_t t = first; t < p.t_end && !*abort_flag; t += gridDim.x) {
-                    const TileInfo ti = decode_tile(te_next);
-                    te_next = fetch_tile(p.tiles, t + gridDim.x, p.t_end);
+                while (!*abort_flag) {
+                    if (!mbar_wait_bounded(&te_full[ws], wph, abort_flag, kWaitLimitNs)) { fail(10); break; }
+                    const TileEntry te = te_slot[ws];
+                    if (te.x == kTileEndX) break;
+                    const TileInfo ti = decode_tile(te);
                     const int row0 = ti.row0, col0 = ti.col0;
                     if (!mbar_wait_bounded(&epi_done[ws], wph, abort_flag, kWaitLimitNs)) { fail(7); break; }
                     const CUtensorMap* mW = p.maps + 3 * (size_t)ti.pair;
@@ -419,8 +460,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
             const int nb = tmem_batches(cf);
             int ws = 0;
             uint32_t wph = 0, aph = 0;
-            for (int64_t t = first; t < p.t_end; t += gridDim.x) {
+            for (;;) {
                 if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+                {
+                    const bool ok = mbar_wait_bounded(&te_full[ws], wph, abort_flag, kWaitLimitNs);
+                    if (!__all_sync(0xffffffffu, ok)) { fail(11); break; }
+                    if (te_slot[ws].x == kTileEndX) break;   // the same for every thread
+                }
                 // 1) sum_e c_e * acc_e for this thread's row, 32 columns,
                 //    one TMEM batch of up to four experts at a time
                 float tot[32];
@@ -464,6 +510,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, 512);
+    }
+    // dynamic schedule: every CTA has taken its last ticket by now; the last
+    // one to get here leaves the counter at zero for the next launch
+    if (p.dyn && threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(p.sched + 1, 1ull) == (unsigned long long)gridDim.x - 1) {
+            atomicExch(p.sched, 0ull);
+            atomicExch(p.sched + 1, 0ull);
+        }
     }
 }
 

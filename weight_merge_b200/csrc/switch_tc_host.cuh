@@ -8,6 +8,7 @@
 #include <cstring>
 
 #include "common.cuh"
+#include "switch_fold.cuh"
 #include "switch_tc.cuh"
 #include "switch_tc2.cuh"
 
@@ -103,6 +104,30 @@ cudaError_t launch_switch_tc(const TcParams& prm, int device, int sm_count, cuda
     const int64_t n = prm.t_end - prm.t_begin;
     const unsigned grid = (unsigned)(n < sm_count ? n : sm_count);
     switch_tc_kernel<KP, BBULK><<<grid, kTcThreads, smem, s>>>(prm);
+    return cudaGetLastError();
+}
+
+// The folded tensor-core switch (ranks <= 8): the fold launch over the
+// weights [w0, w0 + nw) the tiles belong to, then the switch launch, both on
+// `s`.
+inline cudaError_t launch_switch_fold(const TcParams& prm, int64_t w0, int64_t nw, int r,
+                                      int device, int sm_count, cudaStream_t s) {
+    const int smem = (int)FoldConfig::kSmemBytes;
+    static int configured_for = -1;  // device ordinal the attribute was set on
+    if (configured_for != device) {
+        cudaError_t e = cudaFuncSetAttribute(switch_fold_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        configured_for = device;
+    }
+    const unsigned gy = (unsigned)(nw < 65535 ? nw : 65535);
+    fold_operands_kernel<<<dim3(96, gy), kFoldThreads, 0, s>>>(prm.pairs, w0, nw, r, prm.prev,
+                                                               prm.cur, prm.slots, prm.E, prm.s);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int64_t n = prm.t_end - prm.t_begin;
+    const unsigned grid = (unsigned)(n < sm_count ? n : sm_count);
+    switch_fold_kernel<<<grid, kTcThreads, smem, s>>>(prm);
     return cudaGetLastError();
 }
 
