@@ -95,8 +95,13 @@ __device__ __forceinline__ void fold_split(float c, float a, uint16_t& hi, uint1
 __global__ void __launch_bounds__(kFoldThreads) fold_operands_kernel(
     const PairDesc* __restrict__ pairs, int64_t w0, int64_t nw, int r, const int32_t* prev,
     const int32_t* cur, int slots, int E, float s) {
-    Coefs8 cf;
-    if (build_coefs(prev, cur, slots, E, s, cf) != 0) return;  // the switch reports it
+    // the coefficient list, built once per block (the switch reports bad routes)
+    __shared__ Coefs8 s_cf;
+    __shared__ int s_status;
+    if (threadIdx.x == 0) s_status = build_coefs(prev, cur, slots, E, s, s_cf);
+    __syncthreads();
+    if (s_status != 0) return;
+    const Coefs8 cf = s_cf;
     const int npairs = (cf.n + 1) >> 1;
     if (npairs == 0) return;
     const int tid = threadIdx.x;
