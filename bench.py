@@ -80,16 +80,24 @@ KERNEL_SOURCES = {
 
 
 def kernel_source_hash(kernel_name="switch_tc_kernel"):
-    """sha256 over the sources of one kernel and the ABI header (identifies the
-    code an ncu capture was taken on)."""
+    """sha256 over the code of one kernel's sources and the ABI header
+    (identifies the code an ncu capture was taken on).  Comments and
+    whitespace are left out, so a documentation edit keeps the figures while
+    any change to the code voids them."""
     import hashlib
+    import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "weight_merge_b200", "csrc")
     files = [os.path.join(csrc, f) for f in KERNEL_SOURCES[kernel_name]]
     for f in files + [os.path.join(ROOT, "include", "adafuse.h")]:
-        with open(f, "rb") as fh:
-            h.update(os.path.basename(f).encode())
-            h.update(fh.read())
+        with open(f, encoding="utf-8") as fh:
+            text = fh.read()
+        # strip comments (string literals in these files hold no comment markers)
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        text = " ".join(text.split())
+        h.update(os.path.basename(f).encode())
+        h.update(text.encode())
     return h.hexdigest()
 
 

@@ -206,8 +206,9 @@ ADAFUSE_API int adafuse_switch_batch_layers(adafuse_ctx* ctx, int32_t layer_begi
  * otherwise.  With ADAFUSE_KERNEL_TCGEN05_FOLD every switch, re-base or layer
  * range is two launches on the stream: the fold of c_e * A_e for the route's
  * experts into a context-owned buffer (at most 4 pairs of experts x 12 KB per
- * 128 columns of every weight, allocated at create for ranks <= 8), then the
- * switch.  Host-only, no device work. */
+ * 128 columns of every weight, allocated at create for ranks <= 8; when that
+ * allocation fails the context is created without it and this kernel returns
+ * UNSUPPORTED_SHAPE), then the switch.  Host-only, no device work. */
 ADAFUSE_API int adafuse_set_switch_kernel(adafuse_ctx* ctx, int kernel);
 
 /* The kernel adafuse_switch_topk and adafuse_switch_topk_layers launch: the

@@ -345,17 +345,25 @@ int adafuse_create(adafuse_ctx** out, const adafuse_desc* desc, int device) {
     }
     // ranks up to 8: room for the folded operand of up to four expert pairs
     // per 128-column block of every weight (written by each folded switch)
+    // (optional: without the room the context runs the other kernels, and AUTO
+    // gives in-place top-k switches to the four-accumulator kernel)
     if (desc->rank <= 8 && tc_kp_for(desc->rank) != 0) {
         size_t total = 0;
         for (const PairDesc& pd : pairs) total += fold_bytes_for(pd.in);
-        if ((e = cudaMalloc(&c->d_fold, total)) != cudaSuccess)
+        e = cudaMalloc(&c->d_fold, total);
+        if (e == cudaErrorMemoryAllocation) {
+            (void)cudaGetLastError();  // clear it; the context goes on without the buffer
+            c->d_fold = nullptr;
+        } else if (e != cudaSuccess) {
             return fail(e, "cudaMalloc(folded operands)");
-        size_t off = 0;
-        for (PairDesc& pd : pairs) {
-            pd.Af = c->d_fold + off / 2;
-            off += fold_bytes_for(pd.in);
+        } else {
+            size_t off = 0;
+            for (PairDesc& pd : pairs) {
+                pd.Af = c->d_fold + off / 2;
+                off += fold_bytes_for(pd.in);
+            }
+            c->h_pairs = pairs;
         }
-        c->h_pairs = pairs;
     }
     if ((e = cudaMalloc(&c->d_pairs, sizeof(PairDesc) * pairs.size())) != cudaSuccess)
         return fail(e, "cudaMalloc(pairs)");
