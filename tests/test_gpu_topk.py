@@ -279,13 +279,17 @@ def test_rebase_topk_matches_oracle(kernel, r):
                               model.cfg.scale, None, route4_tuple(r_np, t))
 
 
-def test_switch_topk_llama2_7b_shape_sampled():
+@pytest.mark.parametrize("kernel,runs", [(Bnd.ADAFUSE_KERNEL_AUTO, TF), (TC, TC)])
+def test_switch_topk_llama2_7b_shape_sampled(kernel, runs):
     """The 7B shape (E = 8, r = 8) with top-4 routes from the router: every
-    in-place switch touches up to 8 experts (two TMEM batches)."""
+    in-place switch touches up to 8 experts.  AUTO sums them in the folded
+    kernel's one accumulator (the launch the benchmark times); the
+    four-accumulator kernel takes two TMEM batches per tile."""
     cfg = wl.CONFIGS["7b"]
     torch.cuda.empty_cache()
     model = wl.make_model(cfg, device="cuda")
-    sw = switcher(model)
+    sw = switcher(model, kernel)
+    assert sw.topk_kernel == runs
     A_h, B_h = [bits(a) for a in model.A], [bits(b) for b in model.B]
     T, k = 3, 4
     h = wl.make_hidden(cfg, T=T, device="cuda")
