@@ -26,7 +26,9 @@
  * Numerics: W is bf16; each W element is updated as
  *   W <- bf16_round_nearest_even(float(W) + dW)
  * with dW = sum_e c_e * (B_e A_e), the products accumulated in fp32 and the
- * per-expert coefficients c_e = s*(g_cur(e) - g_prev(e)) applied in fp32.
+ * per-expert coefficients c_e = s*(g_cur(e) - g_prev(e)) applied in fp32
+ * (the folded kernel instead carries c_e * A_e as three bf16 terms that
+ * reproduce it to about 2^-24 of its size, one fp32 rounding's worth).
  * One rounding per element per switch.  s = alpha / rank.
  *
  * Layouts (all row-major, all device memory unless stated):
