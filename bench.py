@@ -63,7 +63,13 @@ def parse():
     ap.add_argument("--schedule", choices=["dynamic", "static"], default="dynamic",
                     help="tile schedule of the single-CTA tensor-core kernel")
     ap.add_argument("--no-layerwise", action="store_true",
-                    help="skip the per-layer-launch CUDA graph context figure")
+                    help="skip the per-layer-launch context figures (graph, per-layer routing)")
+    ap.add_argument("--no-pipelined", action="store_true",
+                    help="skip the switch pipelined against a stand-in forward")
+    ap.add_argument("--configs", default="7b-r64,13b,l3-8b",
+                    help="further workloads timed after the headline one (comma list, '' = none)")
+    ap.add_argument("--config-steps", type=int, default=12,
+                    help="timed switches per further workload (at least 10)")
     return ap.parse_args()
 
 
@@ -422,6 +428,259 @@ def reduce_over_ranks(total_ms, n_units, world, device="cpu"):
     return float(mx[0]), float(sm[0])
 
 
+def moving_steps(r_np, seq, prev_t, rebase=False):
+    """For each token t of ``seq`` (the first switch goes prev_t -> seq[0],
+    then token to token): True when that switch moves W.  An in-place switch
+    between bitwise-equal routes is the identity and moves no W bytes; a
+    re-base always writes W.  ``r_np`` must hold the routes the loop used."""
+    import numpy as np
+    out = []
+    p = prev_t
+    for t in seq:
+        out.append(bool(rebase or p is None or not np.array_equal(r_np[p], r_np[t])))
+        p = t
+    return out
+
+
+def e2e_leg(seq, prev_t, run_step, start, stop, read_routes, rebase=False):
+    """The end-to-end loop: ``run_step(prev, t)`` issues one step (host->device
+    copy of the token's input, pre-gate, switch, device->host copy of its
+    route); ``start`` / ``stop`` bracket the loop on the device (``stop``
+    synchronises and returns ms).  The routes are read back AFTER the loop, so
+    the count of W-moving switches describes the routes this loop computed.
+    Returns (ms, moving flags, the token W carries afterwards)."""
+    start()
+    pe = prev_t
+    for t in seq:
+        run_step(pe, t)
+        pe = t
+    ms = stop()
+    return ms, moving_steps(read_routes(), seq, prev_t, rebase), pe
+
+
+KERNEL_NAMES = {1: "switch_mma_kernel", 2: "switch_tc_kernel", 3: "switch_tc2_kernel",
+                4: "switch_fold_kernel"}
+
+
+def route_buffer(cfg, T, topk, device):
+    """Route records of a workload whose switch sequence is synthesised
+    (``share_one`` / ``zipf``), or None when the router makes them."""
+    import numpy as np
+    import torch
+    from weight_merge_b200 import workloads as wl
+    if cfg.route_mode == "router":
+        return None
+    idx, gate = wl.synth_routes(cfg, T=T)
+    width = 8 if topk else 4
+    buf = np.zeros((T, width), dtype=np.int32)
+    half = width // 2
+    if topk:
+        buf[:, :half] = -1
+    buf[:, :2] = idx
+    g = np.zeros((T, half), dtype=np.float32)
+    g[:, :2] = gate
+    buf[:, half:] = g.view(np.int32)
+    return torch.from_numpy(buf).to(device)
+
+
+def percentile(xs, q):
+    s = sorted(xs)
+    return s[min(len(s) - 1, int(q * len(s)))]
+
+
+def config_leg(name, args, dev, stream, peak, peak_kind):
+    """One more workload of the set, switch latency only: the model is built,
+    its route sequence made (router over its hidden states, or synthesised),
+    then 3 warm-up and ``args.config_steps`` timed switches, with CUDA events
+    around each launch on the launching stream.  Identity switches (prev ==
+    cur bitwise) are timed apart and kept out of the roofline."""
+    import torch
+    from weight_merge_b200 import binding as B
+    from weight_merge_b200 import workloads as wl
+
+    cfg = wl.CONFIGS[name]
+    sh = stream.cuda_stream
+    model = wl.make_model(cfg, device="cuda")
+    sw = B.Switcher(model.W, model.A, model.B, cfg.n_layers, len(cfg.targets), cfg.n_experts,
+                    cfg.rank, cfg.alpha, device=dev, names=[t.name for t in cfg.targets])
+    try:
+        kind = sw.kernel
+        T = cfg.n_tokens
+        routes = route_buffer(cfg, T, False, "cuda")
+        if routes is None:
+            h = wl.make_hidden(cfg, T=T, device="cuda")
+            routes = torch.zeros((T, 4), dtype=torch.int32, device="cuda")
+            sw.pregate(h, model.Wr, routes, sh)     # a token's route does not depend on its batch
+            del h
+        torch.cuda.synchronize()
+        r_np = routes.cpu().numpy()
+        warm, n = 3, max(10, args.config_steps)
+        seq = [k % T for k in range(warm + n)]
+        flags = moving_steps(r_np, seq, None)
+        ptr = B.Switcher.route_ptr
+        for k in range(warm):
+            sw.switch(ptr(routes, None if k == 0 else seq[k - 1]), ptr(routes, seq[k]), sh)
+        torch.cuda.synchronize()
+        assert sw.status(sh) == 0
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(n)]
+        with ClockSampler(dev) as clk:
+            torch.cuda.synchronize()
+            clk.mark_start()
+            for k in range(n):
+                i = warm + k
+                ev[k][0].record(stream)
+                sw.switch(ptr(routes, seq[i - 1]), ptr(routes, seq[i]), sh)
+                ev[k][1].record(stream)
+            torch.cuda.synchronize()
+            clk.mark_end()
+        assert sw.status(sh) == 0
+        ms = [a.elapsed_time(b) for a, b in ev]
+        real = [x for x, f in zip(ms, flags[warm:]) if f]
+        ident = [x for x, f in zip(ms, flags[warm:]) if not f]
+        w_bytes = cfg.w_bytes_per_switch()
+        achieved = w_bytes / (sum(real) / len(real) / 1e3) / 1e9
+        kname = KERNEL_NAMES[kind]
+        cpu = None
+        if not args.no_cpu_baseline:
+            gbs, threads, desc, _dt, _el = oracle_rate(cfg, target_s=3.0)
+            cpu = {"value": round(gbs, 5), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                   "sample": desc}
+        return {
+            "workload": workload_label(cfg, T),
+            "route_source": "router" if cfg.route_mode == "router" else f"synthesised ({cfg.route_mode})",
+            "w_bytes_per_switch": w_bytes,
+            "timed_switches": n,
+            "switch_ms_p50": round(percentile(real, 0.5), 4),
+            "switch_ms_p90": round(percentile(real, 0.9), 4),
+            "switches_per_s": round(n / (sum(ms) / 1e3), 3),
+            "identity_steps": len(ident),
+            "identity_switch_ms_p50": round(percentile(ident, 0.5), 5) if ident else None,
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                         "unit": "GB/s", "frac": round(achieved / peak, 4),
+                         "peak_kind": peak_kind, "traffic": profiled_traffic(kname, cfg.name),
+                         "kernel": kname},
+            "cpu_baseline": cpu,
+            "clocks": clk.summary(),
+        }
+    finally:
+        sw.close()
+        del sw, model
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+
+
+def layerwise_dynamic(sw, model, cfg, stream, reps=6):
+    """Layer-wise dynamic routing built from this library's own kernels, the
+    pattern the pages measure AdaFuse against: every layer makes its own
+    routing decision (one pre-gate launch per layer, here over a per-layer
+    stand-in hidden state) and switches its own adapters (one layer-range
+    switch launch per layer, not captured in a graph): 2L launches per token
+    against one pre-gate and one fused switch.  Context only; it leaves W on
+    other routes than the headline sequence, so it runs after it."""
+    import torch
+    from weight_merge_b200 import binding as B
+    L = cfg.n_layers
+    T = reps + 2
+    g = torch.Generator(device="cuda").manual_seed(cfg.seed() + 31)
+    hl = torch.empty((L, T, cfg.d), dtype=torch.float32, device="cuda").normal_(0.0, 1.0, generator=g)
+    rl = torch.zeros((L, T, 4), dtype=torch.int32, device="cuda")
+    sh = stream.cuda_stream
+    ptr = B.Switcher.route_ptr
+
+    def step(t):
+        for layer in range(L):
+            sw.pregate(hl[layer, t:t + 1], model.Wr, rl[layer, t:t + 1], sh)
+            sw.switch_layers(layer, 1, ptr(rl[layer], t - 1) if t > 0 else None,
+                             ptr(rl[layer], t), sh)
+    step(0)
+    step(1)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(reps)]
+    for i in range(reps):
+        ev[i][0].record(stream)
+        step(2 + i)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    assert sw.status(sh) == 0
+    ms = statistics.median(a.elapsed_time(b) for a, b in ev)
+    del hl, rl
+    return {"launches_per_step": 2 * L, "ms_per_step": round(ms, 4), "steps": reps,
+            "kind": "per-layer pre-gate + per-layer switch launch (this library's kernels, "
+                    "no graph); context only"}
+
+
+def pipelined_forward(sw, model, cfg, routes, t_a, t_b, stream, reps=6):
+    """The switch pipelined against a decode forward, layer by layer: a side
+    stream switches layer l (one layer-range launch) and records an event;
+    the main stream waits for it and runs layer l's forward while the side
+    stream switches layer l+1.  The forward here is a stand-in for the
+    caller's decoder (one torch GEMV per targeted weight of the layer, bf16,
+    cuBLAS), not part of this library.  Timed against the serial order (one
+    full switch launch, then the whole forward) and the forward alone.  Each
+    repetition switches t_a -> t_b or back, so W ends where it started."""
+    import torch
+    from weight_merge_b200 import binding as B
+    L, nt = cfg.n_layers, len(cfg.targets)
+    g = torch.Generator(device="cuda").manual_seed(cfg.seed() + 53)
+    xs = [torch.empty(t.inn, dtype=torch.float32, device="cuda").normal_(0.0, 1.0, generator=g)
+          .to(torch.bfloat16) for t in cfg.targets]
+    ys = [torch.empty(t.out, dtype=torch.bfloat16, device="cuda") for t in cfg.targets]
+    side = torch.cuda.Stream()
+    ptr = B.Switcher.route_ptr
+    pair = [(t_a, t_b), (t_b, t_a)]
+    lev = [torch.cuda.Event() for _ in range(L)]
+
+    def forward_layer(layer):
+        for k in range(nt):
+            torch.mv(model.W[layer * nt + k], xs[k], out=ys[k])
+
+    def serial(i):
+        a, b = pair[i % 2]
+        sw.switch(ptr(routes, a), ptr(routes, b), stream.cuda_stream)
+        for layer in range(L):
+            forward_layer(layer)
+
+    def forward_only(i):
+        for layer in range(L):
+            forward_layer(layer)
+
+    def pipelined(i):
+        a, b = pair[i % 2]
+        side.wait_stream(stream)           # the previous forward is done with W
+        for layer in range(L):
+            sw.switch_layers(layer, 1, ptr(routes, a), ptr(routes, b), side.cuda_stream)
+            lev[layer].record(side)
+        for layer in range(L):
+            stream.wait_event(lev[layer])
+            forward_layer(layer)
+
+    out = {}
+    with torch.cuda.stream(stream):
+        for name, fn in (("serial", serial), ("pipelined", pipelined), ("forward_only", forward_only)):
+            fn(0)
+            fn(1)
+            torch.cuda.synchronize()
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(reps)]
+            for i in range(reps):
+                ev[i][0].record(stream)
+                fn(i)
+                ev[i][1].record(stream)
+            torch.cuda.synchronize()
+            out[name] = statistics.median(a.elapsed_time(b) for a, b in ev)
+    assert sw.status(stream.cuda_stream) == 0
+    hidden = (out["serial"] - out["pipelined"]) / out["forward_only"] if out["forward_only"] else None
+    return {"serial_ms": round(out["serial"], 4), "pipelined_ms": round(out["pipelined"], 4),
+            "forward_only_ms": round(out["forward_only"], 4),
+            "speedup": round(out["serial"] / out["pipelined"], 4),
+            "forward_hidden_frac": round(hidden, 4) if hidden is not None else None,
+            "switch_launches": L, "forward_gemvs": L * nt, "reps": reps,
+            "kind": "side-stream layer-range switches ordered by events against a stand-in "
+                    "GEMV forward (torch, the caller's code); context only"}
+
+
 def run_ours(args):
     import numpy as np
     import torch
@@ -455,10 +714,7 @@ def run_ours(args):
                     else B.ADAFUSE_SCHEDULE_STATIC)
     # the kernel this run's switches launch (in-place top-k calls have their own choice)
     kind = sw.topk_kernel if (args.top_k != 2 and args.mode != "rebase") else sw.kernel
-    kernel_name = {B.ADAFUSE_KERNEL_MMA_SYNC: "switch_mma_kernel",
-                   B.ADAFUSE_KERNEL_TCGEN05: "switch_tc_kernel",
-                   B.ADAFUSE_KERNEL_TCGEN05_PAIR: "switch_tc2_kernel",
-                   B.ADAFUSE_KERNEL_TCGEN05_FOLD: "switch_fold_kernel"}[kind]
+    kernel_name = KERNEL_NAMES[kind]
     # the folded kernel's switch is two launches (fold, then switch); the
     # events around a switch cover both
     launches_per_switch = 2 if kind == B.ADAFUSE_KERNEL_TCGEN05_FOLD else 1
@@ -468,7 +724,13 @@ def run_ours(args):
     T = cfg.n_tokens
     h = wl.make_hidden(cfg, T=T, device="cuda")
     topk = args.top_k != 2
-    routes = torch.zeros((T, 8 if topk else 4), dtype=torch.int32, device="cuda")
+    width = 8 if topk else 4
+    # routes: the router's output for router-driven workloads; otherwise the
+    # workload's synthesised sequence (the router still runs every step, into
+    # its own buffer, so the step costs what a decode step costs)
+    synth = route_buffer(cfg, T, topk, "cuda")
+    gated = torch.zeros((T, width), dtype=torch.int32, device="cuda")
+    routes = gated if synth is None else synth
     rptr = B.Switcher.route4_ptr if topk else B.Switcher.route_ptr
 
     def pregate(hh, r_rows):
@@ -492,7 +754,7 @@ def run_ours(args):
 
     def step(k, prev_t):
         t = k % T
-        pregate(h[t:t + 1], routes[t:t + 1])
+        pregate(h[t:t + 1], gated[t:t + 1])
         do_switch(prev_t, t)
         return t
 
@@ -502,6 +764,7 @@ def run_ours(args):
         prev_t = step(k, prev_t)
     torch.cuda.synchronize()
     assert sw.status(sh) == 0
+    first_prev = prev_t
 
     # timed region: K steps, events around every switch launch for the roofline
     n_ev = args.steps
@@ -510,16 +773,15 @@ def run_ours(args):
     st_start = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
     t_begin = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
+    seq = [(args.warmup + k) % T for k in range(args.steps)]
     with ClockSampler(dev) as clk:
         barrier()
         torch.cuda.synchronize()
         clk.mark_start()
         t_begin.record(stream)
-        for k in range(args.steps):
-            kk = args.warmup + k
-            t = kk % T
+        for k, t in enumerate(seq):
             st_start[k].record(stream)
-            pregate(h[t:t + 1], routes[t:t + 1])
+            pregate(h[t:t + 1], gated[t:t + 1])
             sw_start[k].record(stream)
             do_switch(prev_t, t)
             sw_end[k].record(stream)
@@ -535,14 +797,10 @@ def run_ours(args):
     step_ms = [st_start[k].elapsed_time(st_start[k + 1]) for k in range(n_ev - 1)]
     step_ms.append(st_start[-1].elapsed_time(t_end))
 
-    # identity steps (prev == cur bit-identical) move no W bytes
+    # identity steps (prev == cur bit-identical) move no W bytes; the routes
+    # are read after the loop that computed them
     r_np = routes.cpu().numpy()
-    real = []
-    p = (args.warmup - 1) % T if args.warmup > 0 else None
-    for k in range(args.steps):
-        t = (args.warmup + k) % T
-        real.append(bool(rebase or p is None or not np.array_equal(r_np[p], r_np[t])))
-        p = t
+    real = moving_steps(r_np, seq, first_prev, rebase)
     n_real = sum(real)
     # the roofline averages the switches that move W; identity switches are
     # reported on their own
@@ -552,42 +810,45 @@ def run_ours(args):
     max_ms, all_real = reduce_over_ranks(total_ms, n_real, world, device="cuda")
     value = all_real * w_bytes / (max_ms / 1000.0) / 1e9
 
-    # e2e through the public API with host buffers
+    # e2e through the public API with host buffers: each step copies the
+    # token's hidden state from pinned host memory, pre-gates, switches and
+    # copies the token's route record back
     e2e = None
     last_t = prev_t                  # the route W currently carries
     if not args.no_e2e:
         h_host = h.cpu().pin_memory()
-        r_host = torch.zeros((1, routes.shape[1]), dtype=torch.int32).pin_memory()
+        r_host = torch.zeros((1, width), dtype=torch.int32).pin_memory()
         h_dev = torch.empty((1, cfg.d), dtype=torch.float32, device="cuda")
         ev0 = torch.cuda.Event(enable_timing=True)
         ev1 = torch.cuda.Event(enable_timing=True)
-        barrier()
-        torch.cuda.synchronize()
-        ev0.record(stream)
-        pe = prev_t
-        for k in range(args.steps):
-            t = (args.warmup + args.steps + k) % T
+
+        def run_step(pe, t):
             h_dev.copy_(h_host[t:t + 1], non_blocking=True)
-            pregate(h_dev, routes[t:t + 1])
+            pregate(h_dev, gated[t:t + 1])
             do_switch(pe, t)
             r_host.copy_(routes[t:t + 1], non_blocking=True)
-            pe = t
-        last_t = pe
-        ev1.record(stream)
-        torch.cuda.synchronize()
-        barrier()
-        e_ms = ev0.elapsed_time(ev1)
-        e_real = 0
-        pp = prev_t
-        for k in range(args.steps):
-            t = (args.warmup + args.steps + k) % T
-            if rebase or pp is None or not np.array_equal(r_np[pp], r_np[t]):
-                e_real += 1
-            pp = t
-        e_max, e_units = reduce_over_ranks(e_ms, e_real, world, device="cuda")
+
+        def start():
+            barrier()
+            torch.cuda.synchronize()
+            ev0.record(stream)
+
+        def stop():
+            ev1.record(stream)
+            torch.cuda.synchronize()
+            barrier()
+            return ev0.elapsed_time(ev1)
+
+        e_seq = [(args.warmup + args.steps + k) % T for k in range(args.steps)]
+        e_ms, e_flags, last_t = e2e_leg(e_seq, prev_t, run_step, start, stop,
+                                        lambda: routes.cpu().numpy(), rebase)
+        assert sw.status(sh) == 0
+        e_max, e_units = reduce_over_ranks(e_ms, sum(e_flags), world, device="cuda")
         e2e = {"value": round(e_units * w_bytes / (e_max / 1000) / 1e9, 2),
                "unit": "GB/s", "h2d_bytes_per_step": cfg.d * 4,
-               "d2h_bytes_per_step": 4 * routes.shape[1]}
+               "d2h_bytes_per_step": 4 * width, "moving_switches": int(sum(e_flags)),
+               "steps": args.steps, "ms_per_step": round(e_max / args.steps, 4)}
+        r_np = routes.cpu().numpy()
 
     # the router alone on a batch of tokens (the Llama-3-8B-shaped router
     # batch: T=4096, d=4096, E=8): an HBM-bound GEMV over h
@@ -610,22 +871,31 @@ def run_ours(args):
         torch.cuda.synchronize()
         rms = [a.elapsed_time(b) for a, b in zip(ev0, ev1)]
         r_ms = statistics.median(rms)
+        # one decode token: the launch a decode step makes
+        h1 = hr[:1].contiguous()
+        d0 = [torch.cuda.Event(enable_timing=True) for _ in range(20)]
+        d1 = [torch.cuda.Event(enable_timing=True) for _ in range(20)]
+        for i in range(20):
+            d0[i].record(stream)
+            sw.pregate(h1, model.Wr, rr[:1], sh)
+            d1[i].record(stream)
+        torch.cuda.synchronize()
+        dec_ms = statistics.median(a.elapsed_time(b) for a, b in zip(d0, d1))
         del flush
         r_bytes = Tr * cfg.d * 4 + cfg.d * cfg.n_experts * 4 + Tr * 16
         router = {"tokens": Tr, "d": cfg.d, "experts": cfg.n_experts,
                   "ms_p50": round(r_ms, 5), "tokens_per_s": round(Tr / (r_ms / 1e3)),
                   "hbm_gbs": round(r_bytes / (r_ms / 1e3) / 1e9, 1),
                   "frac_of_peak": round(r_bytes / (r_ms / 1e3) / 1e9 / measured_peaks()[0], 4),
-                  "l2": "flushed (256 MB write) before each timed launch"}
+                  "decode_token_ms_p50": round(dec_ms, 5),
+                  "l2": "flushed (256 MB write) before each timed batch launch"}
         del hr, rr
 
-    # context only, never the product path: the same switch as one cuBLAS
-    # addmm_ launch per (layer, target) weight, W += (B_cat * c) @ A_cat in
-    # bf16, the unfused launch pattern the pages contrast with one fused
-    # launch.  Operands are gathered and scaled outside the timed region; it
-    # runs last because it modifies W.
+    # context figures (never the product path), each after the headline
+    # sequence because they move W off it
+    solo = rank == 0 and world == 1
     layerwise = None
-    if rank == 0 and world == 1 and not args.no_layerwise and not rebase and not topk:
+    if solo and not args.no_layerwise and not rebase and not topk:
         layerwise = layerwise_graph(sw, cfg, routes, r_np, last_t if last_t is not None else 0,
                                     stream)
         if layerwise is not None:
@@ -634,21 +904,35 @@ def run_ours(args):
                 statistics.mean(sw_real) / layerwise["ms"], 4)
         assert sw.status(sh) == 0
 
+    pipelined = None
+    if solo and not args.no_pipelined and not rebase and not topk and last_t is not None:
+        other = next((t for t in range(T) if not np.array_equal(r_np[t], r_np[last_t])), None)
+        if other is not None:
+            pipelined = pipelined_forward(sw, model, cfg, routes, last_t, other, stream)
+
+    per_layer_routing = None
+    if solo and not args.no_layerwise and not rebase and not topk:
+        per_layer_routing = layerwise_dynamic(sw, model, cfg, stream)
+        fused = statistics.median(step_ms)
+        per_layer_routing["fused_step_ms_p50"] = round(fused, 4)
+        per_layer_routing["vs_fused_step"] = round(per_layer_routing["ms_per_step"] / fused, 4)
+
     torch_base = None
-    if rank == 0 and world == 1 and not args.no_torch_baseline and not rebase and T > 1:
+    if solo and not args.no_torch_baseline and not rebase and T > 1:
         torch_base = torch_addmm_baseline(model, cfg, r_np, 0, 1, stream)
 
     peak, peak_kind = measured_peaks()
     sw_avg = statistics.mean(sw_real)
     achieved = w_bytes / (sw_avg / 1000.0) / 1e9
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if solo and not args.no_cpu_baseline:
         gbs, threads, desc, dt, elems = oracle_rate(cfg, target_s=10.0)
         cpu = {"value": round(gbs, 5), "unit": "GB/s", "cores": threads, "kind": "oracle",
                "sample": desc}
+    copy_gbs = same_gpu_copy_gbs() if rank == 0 else None
 
+    line = None
     if rank == 0:
-        copy_gbs = same_gpu_copy_gbs()
         sw_sorted = sorted(sw_real)
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
@@ -662,6 +946,7 @@ def run_ours(args):
                 "l2": "inputs larger than L2 (W read+write per switch >> 126 MB), no flush",
                 "parallelism": f"replicas x{world}",
                 "mode": args.mode,
+                "route_source": "router" if synth is None else f"synthesised ({cfg.route_mode})",
                 "tile_schedule": args.schedule if kind == B.ADAFUSE_KERNEL_TCGEN05 else "static",
             },
             "switch_ms_p50": round(sw_sorted[len(sw_sorted) // 2], 4),
@@ -681,13 +966,27 @@ def run_ours(args):
             "cpu_baseline": cpu,
             "torch_addmm_baseline": torch_base,
             "layerwise_graph": layerwise,
+            "per_layer_routing": per_layer_routing,
+            "pipelined": pipelined,
             "e2e": e2e,
             "gpu_launches": (1 + launches_per_switch) * args.steps,
             "router": router,
             "clocks": clocks,
         }
-        print(json.dumps(line), flush=True)
     sw.close()
+    del sw, model, h, routes, gated, synth
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+    # the other workloads of the set, one at a time (replicas run only the
+    # headline workload)
+    if solo and args.configs:
+        extra = {}
+        for name in [c for c in args.configs.split(",") if c and c != args.config]:
+            extra[name] = config_leg(name, args, dev, stream, peak, peak_kind)
+        line["configs"] = extra
+    if rank == 0:
+        print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
 

@@ -132,7 +132,10 @@ def test_pregate_matches_oracle(T, d, E):
     Wr = torch.randn((d, E), generator=g, device="cuda") * 0.05
     sw = make_switcher(model)
     _, got, amb = check_pregate(sw, h, Wr, E)
-    assert len(amb) <= max(1, T // 50)
+    # tokens whose fp32 pick differs from the fp64 oracle, each checked to lie
+    # inside the fp32 rounding bound; none are expected at these sizes
+    print(f"ambiguous tokens: {len(amb)} of {T}")
+    assert len(amb) <= 1
     if E == 1:
         assert np.all(got[:, 1] == -1)
 
@@ -217,8 +220,8 @@ def test_ragged_shapes_every_rank_class(E, r, kernel):
     lockstep(sw, model, routes_np, routes, steps, all_rows, A_h, B_h)
 
 
-def _small_model(seed=3, E=4, r=8):
-    cfg = wl.custom("s", 3, [("q", 256, 384), ("o", 384, 256)], n_experts=E, rank=r,
+def _small_model(seed=3, E=4, r=8, L=3):
+    cfg = wl.custom("s", L, [("q", 256, 384), ("o", 384, 256)], n_experts=E, rank=r,
                     alpha=2.0 * r, n_tokens=4, d=384)
     return wl.make_model(cfg, device="cuda", seed=seed)
 
@@ -276,6 +279,50 @@ def test_layer_ranges_equal_one_full_switch(kernel, r):
         assert np.array_equal(bits(a), bits(b))
     with pytest.raises(Bnd.AdafuseError):
         s2.switch_layers(2, 2, p(0), p(1), stream())
+
+
+@pytest.mark.parametrize("kernel,r", [(TC, 8), (TC2, 16), (TF, 8), (MMA, 12)])
+def test_pipelined_switch_against_a_forward_equals_one_full_switch(kernel, r):
+    """The switch pipelined against a decode forward: a side stream switches
+    one layer per launch and records an event; the main stream waits for
+    layer l's event and then reads layer l's weights (a stand-in forward,
+    one GEMV per weight) while the side stream switches layer l + 1.  Two
+    tokens in a row, the second side stream waiting for the first forward.
+    W must end bit-identical to one full switch per token, and the forward
+    must have read the switched weights."""
+    m1 = _small_model(seed=19, r=r, L=4)
+    m2 = _small_model(seed=19, r=r, L=4)
+    s1, s2 = make_switcher(m1, kernel), make_switcher(m2, kernel)
+    cfg = m1.cfg
+    L, nt = cfg.n_layers, len(cfg.targets)
+    routes = make_routes(np.array([[0, 1], [2, 3], [3, 0]], np.int32),
+                         np.array([[0.7, 0.3], [0.6, 0.4], [0.55, 0.45]], np.float32))
+    p = lambda t: Bnd.Switcher.route_ptr(routes, t)
+    g = torch.Generator(device="cuda").manual_seed(3)
+    xs = [torch.randn(w.shape[1], generator=g, device="cuda").to(torch.bfloat16)
+          for w in m1.W[:nt]]
+    main = torch.cuda.current_stream()
+    side = torch.cuda.Stream()
+    ev = [torch.cuda.Event() for _ in range(L)]
+    ys = []
+    for prev, cur in [(None, 0), (0, 1), (1, 2)]:
+        s1.switch(p(prev), p(cur), main.cuda_stream)
+        side.wait_stream(main)          # the previous forward is done with W
+        for layer in range(L):
+            s2.switch_layers(layer, 1, p(prev), p(cur), side.cuda_stream)
+            ev[layer].record(side)
+        y = []
+        for layer in range(L):
+            main.wait_event(ev[layer])
+            y += [torch.mv(m2.W[layer * nt + k], xs[k]) for k in range(nt)]
+        ys.append(y)
+    torch.cuda.synchronize()
+    assert s1.status(stream()) == 0 and s2.status(stream()) == 0
+    for a, b in zip(m1.W, m2.W):
+        assert np.array_equal(bits(a), bits(b))
+    # the last token's forward read the fully switched weights
+    for i, y in enumerate(ys[-1]):
+        torch.testing.assert_close(y, torch.mv(m1.W[i], xs[i % nt]), rtol=0, atol=0)
 
 
 @pytest.mark.parametrize("r", [8, 4, 16])
