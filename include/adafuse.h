@@ -44,8 +44,9 @@
  * on it is in flight.  The library owns the context, its device-side
  * segment table and its device status word.  The library keeps no copy of W.
  * For ranks below 8 it keeps a zero-padded copy of every B (see
- * adafuse_refresh_adapters); for ranks up to 8 a buffer the folded kernel
- * rewrites from A on every switch (see ADAFUSE_KERNEL_TCGEN05_FOLD).
+ * adafuse_refresh_adapters); for ranks up to 8, once the folded kernel is
+ * first used, a buffer that kernel rewrites from A on every switch (see
+ * adafuse_set_switch_kernel).
  *
  * Errors: every call returns ADAFUSE_OK (0) or a negative code.  Calls that
  * take a stream are asynchronous with respect to the host; host-side
@@ -207,10 +208,16 @@ ADAFUSE_API int adafuse_switch_batch_layers(adafuse_ctx* ctx, int32_t layer_begi
  * ADAFUSE_KERNEL_TCGEN05_FOLD rank <= 8; each returns UNSUPPORTED_SHAPE
  * otherwise.  With ADAFUSE_KERNEL_TCGEN05_FOLD every switch, re-base or layer
  * range is two launches on the stream: the fold of c_e * A_e for the route's
- * experts into a context-owned buffer (at most 4 pairs of experts x 12 KB per
- * 128 columns of every weight, allocated at create for ranks <= 8; when that
- * allocation fails the context is created without it and this kernel returns
- * UNSUPPORTED_SHAPE), then the switch.  Host-only, no device work. */
+ * experts into a context-owned buffer, then the switch.  That buffer holds at
+ * most 4 pairs of experts x 12 KB per 128 columns of every weight (48 KB per
+ * 128 columns; 437 MB at the Llama-2-7B shape) and is allocated on first use:
+ * by this call when it selects ADAFUSE_KERNEL_TCGEN05_FOLD, or by the first
+ * in-place top-k switch that ADAFUSE_KERNEL_AUTO gives to the folded kernel.
+ * That first use synchronises the device and must not be captured into a
+ * CUDA graph (INVALID_ARG, nothing enqueued).  If the allocation fails it
+ * returns OUT_OF_MEMORY and the folded kernel is off for the context (AUTO
+ * then takes ADAFUSE_KERNEL_TCGEN05 for top-k switches).  Selecting any other
+ * kernel is host-only, with no device work. */
 ADAFUSE_API int adafuse_set_switch_kernel(adafuse_ctx* ctx, int kernel);
 
 /* The kernel adafuse_switch_topk and adafuse_switch_topk_layers launch: the
@@ -343,11 +350,13 @@ ADAFUSE_API int adafuse_segment_table(const adafuse_desc* desc, int32_t* entries
  * Scratch: one file-scope static device array of
  * ADAFUSE_NOALLOC_SCRATCH_BYTES (64 KiB), which every GPU that loads this
  * library holds until the process exits.  Each call rewrites it with the
- * weight table of `desc`, so ALL calls share it: two calls whose work
- * overlaps on the GPU (different streams, or threads without ordering)
- * race and may switch the wrong weights.  Calls on one stream are ordered
- * and safe.  The first call on each device also looks up the array's device
- * address (once per device); make that first call before any stream capture.
+ * weight table of `desc`, written on the device by small launches that carry
+ * the table entries as kernel arguments (no host buffer is read after the
+ * call returns), so ALL calls share it: two calls whose work overlaps on the
+ * GPU (different streams, or threads without ordering) race and may switch
+ * the wrong weights.  Calls on one stream are ordered and safe.  The first
+ * call on each device also looks up the array's device address (once per
+ * device); make that first call before any stream capture.
  *
  * Arguments: desc as for adafuse_create (host memory, read during the call
  * only; its device pointers must stay valid until the switch completes);
@@ -357,7 +366,9 @@ ADAFUSE_API int adafuse_segment_table(const adafuse_desc* desc, int32_t* entries
  * Returns ADAFUSE_ERR_UNSUPPORTED_SHAPE when desc has more than
  * ADAFUSE_NOALLOC_MAX_WEIGHTS weights (or a shape adafuse_create rejects),
  * INVALID_ARG / UNSUPPORTED_DEVICE / CUDA otherwise as adafuse_create and
- * adafuse_switch do.  Asynchronous like adafuse_switch. */
+ * adafuse_switch do; every argument is checked before anything is enqueued.
+ * Asynchronous like adafuse_switch: it enqueues ceil(weights / 96) table
+ * launches, the status reset and the switch launch on `stream`. */
 ADAFUSE_API int adafuse_switch_noalloc(const adafuse_desc* desc, const adafuse_route* prev,
                                        const adafuse_route* cur, int32_t* status, void* stream);
 

@@ -24,6 +24,9 @@ pytestmark = pytest.mark.gpu
 MMA, TC, TC2, TF = (Bnd.ADAFUSE_KERNEL_MMA_SYNC, Bnd.ADAFUSE_KERNEL_TCGEN05,
                     Bnd.ADAFUSE_KERNEL_TCGEN05_PAIR, Bnd.ADAFUSE_KERNEL_TCGEN05_FOLD)
 GATE_RTOL = 1e-5
+# tokens whose fp32 pick may differ from the fp64 oracle (each one checked to
+# lie inside the fp32 rounding bound); none are expected at these sizes
+AMBIGUOUS_MAX = 1
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -71,7 +74,8 @@ def test_pregate_topk_matches_oracle(T, d, E, k):
     h_np, Wr_np = h.cpu().numpy(), Wr.cpu().numpy()
     idx_ref, gate_ref, z = oracle.pregate_topk(h_np, Wr_np, k, return_logits=True)
     amb = pregate_topk_consistent(got[:, :k], idx_ref, z, h_np, Wr_np)
-    assert len(amb) <= max(1, T // 50)
+    print(f"ambiguous tokens: {len(amb)} of {T}")
+    assert len(amb) <= AMBIGUOUS_MAX
     match = np.all(got[:, :k] == idx_ref, axis=1)
     gates = got[:, 4:].view(np.float32)
     np.testing.assert_allclose(gates[match, :k], gate_ref[match], rtol=GATE_RTOL, atol=1e-30)
@@ -288,7 +292,15 @@ def test_switch_topk_llama2_7b_shape_sampled(kernel, runs):
     cfg = wl.CONFIGS["7b"]
     torch.cuda.empty_cache()
     model = wl.make_model(cfg, device="cuda")
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
     sw = switcher(model, kernel)
+    created = free0 - torch.cuda.mem_get_info()[0]
+    # the context holds its tile table (8 B per 128 x 128 tile), three tensor
+    # maps and one descriptor per weight; the folded kernel's operand buffer
+    # (437 MB here) waits for the first folded switch
+    table = 8 * 395264 + len(model.W) * (3 * 128 + 64)
+    assert created < table + (16 << 20), created
     assert sw.topk_kernel == runs
     A_h, B_h = [bits(a) for a in model.A], [bits(b) for b in model.B]
     T, k = 3, 4
@@ -306,9 +318,35 @@ def test_switch_topk_llama2_7b_shape_sampled(kernel, runs):
         off = ((i // nt) * 7 + (i % nt) * 13) % 97
         return np.arange(off, out, 97, dtype=np.int64)
     _lockstep(sw, model, routes, [(None, 0), (0, 1), (1, 2)], A_h, B_h, rows_of)
+    if runs == TF:
+        # the first folded switch allocated the buffer
+        assert free0 - torch.cuda.mem_get_info()[0] - created >= 400 << 20
     sw.close()
     del model
     torch.cuda.empty_cache()
+
+
+def test_first_folded_switch_is_refused_inside_graph_capture():
+    """The folded kernel's buffer is allocated by its first use, which may not
+    sit inside stream capture: the call returns INVALID_ARG with nothing
+    enqueued.  Made eagerly afterwards, the same switch matches the oracle."""
+    model = _small(seed=14, r=8)
+    sw = switcher(model)
+    assert sw.topk_kernel == TF
+    routes = make_routes4(np.array([[0, 2, 5, 1]], np.int32),
+                          np.array([[0.4, 0.3, 0.2, 0.1]], np.float32))
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with pytest.raises(Bnd.AdafuseError) as err:
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(graph, stream=side):
+                sw.switch_topk(None, Bnd.Switcher.route4_ptr(routes, 0), side.cuda_stream)
+    assert err.value.code == Bnd.ADAFUSE_ERR_INVALID_ARG
+    del graph
+    torch.cuda.synchronize()
+    A_h, B_h = [bits(a) for a in model.A], [bits(b) for b in model.B]
+    _lockstep(sw, model, routes, [(None, 0)], A_h, B_h)
 
 
 # --------------------------------------------------------------------------
@@ -343,7 +381,8 @@ def test_pregate_topk_odd_sizes_and_many_experts(T, d, E, k):
     h_np, Wr_np = h.cpu().numpy(), Wr.cpu().numpy()
     idx_ref, gate_ref, z = oracle.pregate_topk(h_np, Wr_np, k, return_logits=True)
     amb = pregate_topk_consistent(got[:, :k], idx_ref, z, h_np, Wr_np)
-    assert len(amb) <= max(1, T // 50)
+    print(f"ambiguous tokens: {len(amb)} of {T}")
+    assert len(amb) <= AMBIGUOUS_MAX
     match = np.all(got[:, :k] == idx_ref, axis=1)
     np.testing.assert_allclose(got[match, 4:4 + k].view(np.float32), gate_ref[match],
                                rtol=GATE_RTOL, atol=1e-30)

@@ -41,6 +41,8 @@ struct adafuse_ctx {
     TileEntry* d_blocks = nullptr;
     uint16_t* d_bpad = nullptr;              // rank < 8: B with rows zero-padded to 8
     uint16_t* d_fold = nullptr;              // rank <= 8: folded-coefficient operands
+                                             // (allocated on first use, see ensure_fold)
+    bool fold_failed = false;                // that allocation failed: the kernel is off
     unsigned long long* d_sched = nullptr;   // [2] ticket counter of the dynamic tile schedule
     int schedule = ADAFUSE_SCHEDULE_DYNAMIC;
     std::vector<int64_t> layer_block_begin;  // [n_layers + 1]
@@ -133,8 +135,61 @@ int64_t walk_blocks(const adafuse_desc* d, Emit&& emit) {
 // tensor maps fetch exactly 8 rows for the single-CTA kernel's layout).
 bool pair_eligible(const adafuse_ctx* c) { return c->tc_kp != 0 && c->rank > 8; }
 
-// The folded kernel takes ranks up to 8 once its operand buffer exists.
-bool fold_eligible(const adafuse_ctx* c) { return c->tc_kp != 0 && c->d_fold != nullptr; }
+// The folded kernel takes ranks up to 8 unless its operand buffer could not
+// be allocated (it is allocated on first use, see ensure_fold).
+bool fold_eligible(const adafuse_ctx* c) {
+    return c->tc_kp != 0 && c->rank <= 8 && !c->fold_failed;
+}
+
+// The folded kernel's operand buffer, allocated on the first call that needs
+// it (adafuse_set_switch_kernel(FOLD), or the first in-place top-k switch that
+// AUTO gives to the folded kernel) rather than at create: a context that
+// never folds pays nothing for it.  Allocating synchronises the device, so
+// the first use may not be captured into a graph (INVALID_ARG then, with
+// nothing enqueued).  An allocation failure turns the kernel off for the
+// context (OUT_OF_MEMORY).
+int ensure_fold(adafuse_ctx* c, cudaStream_t capture_check) {
+    if (c->d_fold != nullptr) return ADAFUSE_OK;
+    if (!fold_eligible(c)) return ADAFUSE_ERR_UNSUPPORTED_SHAPE;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(capture_check, &cs);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamIsCapturing");
+    if (cs != cudaStreamCaptureStatusNone) return ADAFUSE_ERR_INVALID_ARG;
+    size_t total = 0;
+    for (const PairDesc& pd : c->h_pairs) total += fold_bytes_for(pd.in);
+    std::vector<PairDesc> pairs;
+    try {
+        pairs = c->h_pairs;
+    } catch (...) {
+        return ADAFUSE_ERR_OUT_OF_MEMORY;
+    }
+    uint16_t* buf = nullptr;
+    e = cudaMalloc(&buf, total);
+    if (e == cudaErrorMemoryAllocation) {
+        (void)cudaGetLastError();
+        c->fold_failed = true;
+        return ADAFUSE_ERR_OUT_OF_MEMORY;
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(folded operands)");
+    size_t off = 0;
+    for (PairDesc& pd : pairs) {
+        pd.Af = buf + off / 2;
+        off += fold_bytes_for(pd.in);
+    }
+    // the descriptors may be read by work still in flight: replace them once
+    // the device is idle
+    e = cudaDeviceSynchronize();
+    if (e == cudaSuccess)
+        e = cudaMemcpy(c->d_pairs, pairs.data(), sizeof(PairDesc) * pairs.size(),
+                       cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) {
+        cudaFree(buf);
+        return cuda_fail(e, "folded operand descriptors");
+    }
+    c->h_pairs.swap(pairs);
+    c->d_fold = buf;
+    return ADAFUSE_OK;
+}
 
 // Rank < 8: copy every B [E, out, r] into its [E, out, 8] zero-padded slot
 // (the padding columns are zeroed once, at create).
@@ -343,28 +398,6 @@ int adafuse_create(adafuse_ctx** out, const adafuse_desc* desc, int device) {
         if ((e = copy_padded_b(c, nullptr)) != cudaSuccess) return fail(e, "cudaMemcpy2D(padded B)");
         if ((e = cudaDeviceSynchronize()) != cudaSuccess) return fail(e, "padded B");
     }
-    // ranks up to 8: room for the folded operand of up to four expert pairs
-    // per 128-column block of every weight (written by each folded switch)
-    // (optional: without the room the context runs the other kernels, and AUTO
-    // gives in-place top-k switches to the four-accumulator kernel)
-    if (desc->rank <= 8 && tc_kp_for(desc->rank) != 0) {
-        size_t total = 0;
-        for (const PairDesc& pd : pairs) total += fold_bytes_for(pd.in);
-        e = cudaMalloc(&c->d_fold, total);
-        if (e == cudaErrorMemoryAllocation) {
-            (void)cudaGetLastError();  // clear it; the context goes on without the buffer
-            c->d_fold = nullptr;
-        } else if (e != cudaSuccess) {
-            return fail(e, "cudaMalloc(folded operands)");
-        } else {
-            size_t off = 0;
-            for (PairDesc& pd : pairs) {
-                pd.Af = c->d_fold + off / 2;
-                off += fold_bytes_for(pd.in);
-            }
-            c->h_pairs = pairs;
-        }
-    }
     if ((e = cudaMalloc(&c->d_pairs, sizeof(PairDesc) * pairs.size())) != cudaSuccess)
         return fail(e, "cudaMalloc(pairs)");
     if ((e = cudaMalloc(&c->d_tiles, sizeof(TileEntry) * tiles.size())) != cudaSuccess)
@@ -462,8 +495,13 @@ int adafuse_set_switch_kernel(adafuse_ctx* ctx, int kernel) {
     if (kernel == ADAFUSE_KERNEL_TCGEN05 && ctx->tc_kp == 0) return ADAFUSE_ERR_UNSUPPORTED_SHAPE;
     if (kernel == ADAFUSE_KERNEL_TCGEN05_PAIR && !pair_eligible(ctx))
         return ADAFUSE_ERR_UNSUPPORTED_SHAPE;
-    if (kernel == ADAFUSE_KERNEL_TCGEN05_FOLD && !fold_eligible(ctx))
-        return ADAFUSE_ERR_UNSUPPORTED_SHAPE;
+    if (kernel == ADAFUSE_KERNEL_TCGEN05_FOLD) {
+        if (!fold_eligible(ctx)) return ADAFUSE_ERR_UNSUPPORTED_SHAPE;
+        DeviceGuard guard(ctx->device);
+        if (!guard.ok) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
+        const int rc = ensure_fold(ctx, nullptr);
+        if (rc != ADAFUSE_OK) return rc;
+    }
     ctx->kernel = kernel;
     return ADAFUSE_OK;
 }
@@ -589,8 +627,16 @@ int launch_switch(adafuse_ctx* ctx, int32_t layer_begin, int32_t n_layers,
     DeviceGuard guard(ctx->device);
     if (!guard.ok) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const int kind = slots == 4 && !rebase ? adafuse_get_topk_switch_kernel(ctx)
-                                           : adafuse_get_switch_kernel(ctx);
+    int kind = slots == 4 && !rebase ? adafuse_get_topk_switch_kernel(ctx)
+                                     : adafuse_get_switch_kernel(ctx);
+    if (kind == ADAFUSE_KERNEL_TCGEN05_FOLD && ctx->d_fold == nullptr) {
+        const int rc = ensure_fold(ctx, s);
+        if (rc == ADAFUSE_ERR_OUT_OF_MEMORY && ctx->kernel == ADAFUSE_KERNEL_AUTO)
+            kind = slots == 4 && !rebase ? adafuse_get_topk_switch_kernel(ctx)
+                                         : adafuse_get_switch_kernel(ctx);  // AUTO falls back
+        else if (rc != ADAFUSE_OK)
+            return rc;
+    }
     if (kind == ADAFUSE_KERNEL_TCGEN05_PAIR) {
         const int64_t b0 = ctx->layer_block_begin[(size_t)layer_begin];
         const int64_t b1 = ctx->layer_block_begin[(size_t)layer_begin + n_layers];
