@@ -11,10 +11,12 @@
 // buffers is one file-scope static array (kScratchBytes, below), which every
 // GPU that loads the library holds until the process exits.
 //
-// Each call writes the per-weight table into that array, so every call shares
-// it: calls whose work overlaps on the GPU (different streams, or different
-// host threads without ordering) race on it.  Calls on one stream are ordered
-// and safe.  The first call on a device looks up the array's device address
+// Each call writes the per-weight table into that array through a few small
+// launches that carry the entries as kernel arguments (no host staging
+// buffer, no host-to-device copy), so every call shares the array: calls
+// whose work overlaps on the GPU (different streams, or different host
+// threads without ordering) race on it.  Calls on one stream are ordered and
+// safe.  The first call on a device looks up the array's device address
 // (cudaGetSymbolAddress) once for that device; make that first call before
 // any stream capture.
 #include <cuda_runtime.h>
@@ -213,18 +215,28 @@ switch_noalloc_kernel(const Entry* __restrict__ tab, int n_weights, int64_t n_ti
     }
 }
 
-// Host staging for the table (static storage, no heap), guarded by g_mu
-// together with the per-device set-up below.  A pageable cudaMemcpyAsync
-// returns once the source has been staged, so the buffer is free again when
-// the call returns.
+// The table is written on the device by small launches whose arguments carry
+// up to kFillChunk entries each (3.8 KB of a launch's 4 KB argument space).
+constexpr int kFillChunk = 96;
+struct EntryChunk {
+    Entry e[kFillChunk];
+};
+static_assert(sizeof(EntryChunk) + 16 <= 4096, "kernel argument space");
+
+__global__ void fill_table_kernel(Entry* tab, const EntryChunk chunk, int first, int count) {
+    const int i = threadIdx.x;
+    if (i < count) tab[first + i] = chunk.e[i];
+}
+
+// Per-device set-up (the scratch's device address), guarded by g_mu; the
+// mutex is held only while a device is set up, never across GPU work.
 std::mutex g_mu;
-Entry g_host_table[kMaxWeights];
 void* g_scratch_dev[kMaxDevices] = {};
 int g_sm_count[kMaxDevices] = {};
 
 // Once per device, with that device current: the scratch's device address.
-// Caller holds g_mu.
 int setup_device(int dev, void** scratch, int* sms) {
+    std::lock_guard<std::mutex> lk(g_mu);
     if (g_scratch_dev[dev] == nullptr) {
         int major = 0, minor = 0, count = 0;
         cudaError_t e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
@@ -263,7 +275,7 @@ extern "C" int adafuse_switch_noalloc(const adafuse_desc* desc, const adafuse_ro
     static_assert(kMaxWeights == ADAFUSE_NOALLOC_MAX_WEIGHTS, "header limit");
     static_assert(kScratchBytes == ADAFUSE_NOALLOC_SCRATCH_BYTES, "header size");
     if (n > kMaxWeights) return ADAFUSE_ERR_UNSUPPORTED_SHAPE;  // more than the scratch holds
-    std::lock_guard<std::mutex> lk(g_mu);
+    // every argument is checked before anything is enqueued
     int64_t tiles = 0;
     for (int64_t i = 0; i < n; ++i) {
         const adafuse_target& t = desc->targets[i];
@@ -274,13 +286,6 @@ extern "C" int adafuse_switch_noalloc(const adafuse_desc* desc, const adafuse_ro
         if ((reinterpret_cast<uintptr_t>(t.W) | reinterpret_cast<uintptr_t>(t.A) |
              reinterpret_cast<uintptr_t>(t.B)) & 15u)
             return ADAFUSE_ERR_INVALID_ARG;
-        Entry& en = g_host_table[i];
-        en.W = static_cast<uint16_t*>(t.W);
-        en.A = static_cast<const uint16_t*>(t.A);
-        en.B = static_cast<const uint16_t*>(t.B);
-        en.out = (int32_t)t.out;
-        en.in = (int32_t)t.in;
-        en.tile_begin = tiles;
         tiles += ((t.out + kTile - 1) / kTile) * ((t.in + kTile - 1) / kTile);
     }
 
@@ -292,11 +297,30 @@ extern "C" int adafuse_switch_noalloc(const adafuse_desc* desc, const adafuse_ro
     int sms = 0;
     int rc = setup_device(dev, &scratch, &sms);
     if (rc != ADAFUSE_OK) return rc;
+    Entry* tab = static_cast<Entry*>(scratch);
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // the table is rewritten in full by every call; the status output starts at zero
-    e = cudaMemcpyAsync(scratch, g_host_table, sizeof(Entry) * (size_t)n, cudaMemcpyHostToDevice, s);
-    if (e != cudaSuccess) return ADAFUSE_ERR_CUDA;
+    // the table is rewritten in full by every call, in stream order before
+    // the switch launch; the status output starts at zero
+    EntryChunk chunk;
+    int64_t begin = 0;
+    for (int64_t i0 = 0; i0 < n; i0 += kFillChunk) {
+        const int cnt = (int)(n - i0 < kFillChunk ? n - i0 : kFillChunk);
+        for (int j = 0; j < cnt; ++j) {
+            const adafuse_target& t = desc->targets[i0 + j];
+            Entry& en = chunk.e[j];
+            en.W = static_cast<uint16_t*>(t.W);
+            en.A = static_cast<const uint16_t*>(t.A);
+            en.B = static_cast<const uint16_t*>(t.B);
+            en.out = (int32_t)t.out;
+            en.in = (int32_t)t.in;
+            en.tile_begin = begin;
+            begin += ((t.out + kTile - 1) / kTile) * ((t.in + kTile - 1) / kTile);
+        }
+        fill_table_kernel<<<1, kFillChunk, 0, s>>>(tab, chunk, (int)i0, cnt);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return ADAFUSE_ERR_CUDA;
+    }
     if (status != nullptr) {
         e = cudaMemsetAsync(status, 0, sizeof(int32_t), s);
         if (e != cudaSuccess) return ADAFUSE_ERR_CUDA;
@@ -304,7 +328,6 @@ extern "C" int adafuse_switch_noalloc(const adafuse_desc* desc, const adafuse_ro
     if (tiles == 0) return ADAFUSE_OK;
     const int64_t want = (int64_t)sms * 2;
     const unsigned grid = (unsigned)(tiles < want ? tiles : want);
-    const Entry* tab = static_cast<const Entry*>(scratch);
     const int E = desc->n_experts, r = desc->rank;
     const float sc = desc->alpha / (float)desc->rank;
     const int nw = (int)n;
