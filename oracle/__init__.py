@@ -61,6 +61,7 @@ def _load():
         lib.orc_switch_rows_k.argtypes = [P, P, i64, i64, i64, P, P, i32, dbl, i32,
                                           P, P, P, P, P, P]
         lib.orc_pregate_topk.argtypes = [P, i64, i64, P, i32, i32, P, P, P]
+        lib.orc_pregate_batch.argtypes = [P, i64, i64, P, i32, i32, P, P, P]
         lib.orc_num_threads.restype = ctypes.c_int
         lib.orc_set_num_threads.argtypes = [ctypes.c_int]
         _lib = lib
@@ -131,6 +132,29 @@ def pregate_topk(h: np.ndarray, Wr: np.ndarray, k: int, return_logits: bool = Fa
     _load().orc_pregate_topk(_ptr(h), T, d, _ptr(Wr), E, k, _ptr(idx), _ptr(gate), _ptr(z))
     if return_logits:
         return idx, gate, z
+    return idx, gate
+
+
+def pregate_batch(h: np.ndarray, Wr: np.ndarray, k: int = 2, return_logits: bool = False):
+    """One routing decision for a decode batch (a reading beyond the pages'
+    per-token router, see adafuse_oracle.c): the top-k of the tokens' mean
+    logits, gates = their softmax renormalised over the picks.
+
+    h [T, d] fp32 (T >= 1), Wr [d, E] fp32  ->  idx [k] int32, gate [k] fp32
+    (and the fp64 mean logits [E] when ``return_logits``).
+    """
+    assert 1 <= k <= 4
+    h = np.ascontiguousarray(h, dtype=np.float32)
+    Wr = np.ascontiguousarray(Wr, dtype=np.float32)
+    T, d = h.shape
+    d2, E = Wr.shape
+    assert d == d2 and T >= 1
+    idx = np.empty(k, dtype=np.int32)
+    gate = np.empty(k, dtype=np.float32)
+    zbar = np.empty(E, dtype=np.float64)
+    _load().orc_pregate_batch(_ptr(h), T, d, _ptr(Wr), E, k, _ptr(idx), _ptr(gate), _ptr(zbar))
+    if return_logits:
+        return idx, gate, zbar
     return idx, gate
 
 

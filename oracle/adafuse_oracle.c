@@ -179,6 +179,62 @@ void orc_pregate_topk(const float* h, int64_t T, int64_t d, const float* Wr,
     }
 }
 
+/* Batch pre-gating: ONE routing decision for a decode batch of T tokens
+ * that shares one merged weight.  A reading beyond [P2] 2-ga, which makes
+ * one decision per token: a batch whose tokens would pick different experts
+ * can carry only one expert set in W, so the batch's router logits are
+ * averaged and the token rule is applied to the mean:
+ *   z_t,e  = sum_i h[t,i] Wr[i,e]           (each token's logits, fp64)
+ *   zbar_e = (1/T) sum_t z_t,e
+ *   pick j = the largest zbar among the experts not yet picked, lowest
+ *            index among equals, j < k (k in [1, 4]);
+ *   g_j    = softmax(zbar) over all E renormalised over the k picks,
+ *            rounded to fp32.
+ * Slots past E hold idx -1 and gate 0.  idx_out / gate_out are [k]; the
+ * mean logits go to zbar_out ([E]) when it is not NULL.  T >= 1. */
+void orc_pregate_batch(const float* h, int64_t T, int64_t d, const float* Wr,
+                       int32_t E, int32_t k, int32_t* idx_out, float* gate_out,
+                       double* zbar_out) {
+    double* zbar = (double*)calloc((size_t)E, sizeof(double));
+    char* taken = (char*)calloc((size_t)E, 1);
+    for (int64_t t = 0; t < T; ++t)
+        for (int32_t e = 0; e < E; ++e) {
+            double acc = 0.0;
+            for (int64_t i = 0; i < d; ++i)
+                acc += (double)h[t * d + i] * (double)Wr[i * E + e];
+            zbar[e] += acc;
+        }
+    for (int32_t e = 0; e < E; ++e) zbar[e] /= (double)T;
+    int32_t pick[4] = {-1, -1, -1, -1};
+    for (int32_t j = 0; j < k; ++j) {
+        int32_t best = -1;
+        for (int32_t e = 0; e < E; ++e) {
+            if (taken[e]) continue;
+            if (best < 0 || zbar[e] > zbar[best]) best = e;
+        }
+        if (best < 0) break;
+        pick[j] = best;
+        taken[best] = 1;
+    }
+    double zmax = zbar[pick[0]];
+    double denom = 0.0;
+    for (int32_t e = 0; e < E; ++e) denom += exp(zbar[e] - zmax);
+    double p[4] = {0.0, 0.0, 0.0, 0.0}, psum = 0.0;
+    for (int32_t j = 0; j < k; ++j)
+        if (pick[j] >= 0) {
+            p[j] = exp(zbar[pick[j]] - zmax) / denom;
+            psum += p[j];
+        }
+    for (int32_t j = 0; j < k; ++j) {
+        idx_out[j] = pick[j];
+        gate_out[j] = pick[j] >= 0 ? (float)(p[j] / psum) : 0.0f;
+    }
+    if (zbar_out)
+        for (int32_t e = 0; e < E; ++e) zbar_out[e] = zbar[e];
+    free(taken);
+    free(zbar);
+}
+
 /* ---- fused adapter switch ([P1] abstract, [P2] 2-na) -------------------- */
 
 /* The experts a route of `slots` slots names (slots holding -1 are empty).
