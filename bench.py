@@ -611,7 +611,7 @@ def layerwise_dynamic(sw, model, cfg, stream, reps=6):
                     "no graph); context only"}
 
 
-def pipelined_forward(sw, model, cfg, routes, t_a, t_b, stream, reps=6):
+def pipelined_forward(sw, model, cfg, routes, t_a, t_b, stream, reps=6, caps=(0, 128, 112)):
     """The switch pipelined against a decode forward, layer by layer: a side
     stream switches layer l (one layer-range launch) and records an event;
     the main stream waits for it and runs layer l's forward while the side
@@ -656,29 +656,43 @@ def pipelined_forward(sw, model, cfg, routes, t_a, t_b, stream, reps=6):
             stream.wait_event(lev[layer])
             forward_layer(layer)
 
+    def timed(fn):
+        fn(0)
+        fn(1)
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(reps)]
+        for i in range(reps):
+            ev[i][0].record(stream)
+            fn(i)
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        return statistics.median(a.elapsed_time(b) for a, b in ev)
+
     out = {}
     with torch.cuda.stream(stream):
-        for name, fn in (("serial", serial), ("pipelined", pipelined), ("forward_only", forward_only)):
-            fn(0)
-            fn(1)
-            torch.cuda.synchronize()
-            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                  for _ in range(reps)]
-            for i in range(reps):
-                ev[i][0].record(stream)
-                fn(i)
-                ev[i][1].record(stream)
-            torch.cuda.synchronize()
-            out[name] = statistics.median(a.elapsed_time(b) for a, b in ev)
+        out["serial"] = timed(serial)
+        out["forward_only"] = timed(forward_only)
+        # the pipelined schedule with the switch's grid capped, so that the
+        # forward's kernels find free SMs beside it (0 = no cap)
+        for cap in caps:
+            sw.set_max_ctas(cap)
+            out[f"pipelined_cap{cap}"] = timed(pipelined)
+        sw.set_max_ctas(0)
     assert sw.status(stream.cuda_stream) == 0
-    hidden = (out["serial"] - out["pipelined"]) / out["forward_only"] if out["forward_only"] else None
-    return {"serial_ms": round(out["serial"], 4), "pipelined_ms": round(out["pipelined"], 4),
+    best_cap = min(caps, key=lambda c: out[f"pipelined_cap{c}"])
+    best = out[f"pipelined_cap{best_cap}"]
+    hidden = (out["serial"] - best) / out["forward_only"] if out["forward_only"] else None
+    return {"serial_ms": round(out["serial"], 4),
+            "pipelined_ms": {str(c): round(out[f"pipelined_cap{c}"], 4) for c in caps},
+            "best_switch_ctas": best_cap or None,
             "forward_only_ms": round(out["forward_only"], 4),
-            "speedup": round(out["serial"] / out["pipelined"], 4),
+            "speedup": round(out["serial"] / best, 4),
             "forward_hidden_frac": round(hidden, 4) if hidden is not None else None,
             "switch_launches": L, "forward_gemvs": L * nt, "reps": reps,
             "kind": "side-stream layer-range switches ordered by events against a stand-in "
-                    "GEMV forward (torch, the caller's code); context only"}
+                    "GEMV forward (torch, the caller's code), switch grid capped at the given "
+                    "CTA counts (0 = every SM); context only"}
 
 
 def run_ours(args):

@@ -84,8 +84,9 @@ extern "C" {
 /* ---- device status word bits (adafuse_get_device_status) ---------------- */
 #define ADAFUSE_STATUS_BAD_EXPERT   0x1   /* a route held an index outside [-1, E) */
 #define ADAFUSE_STATUS_BAD_GATE     0x2   /* a route held a non-finite gate on a used slot */
-#define ADAFUSE_STATUS_TIMEOUT      0x4   /* a bounded wait inside the switch kernel gave up
-                                             (the switch is then incomplete) */
+#define ADAFUSE_STATUS_TIMEOUT      0x4   /* a bounded wait inside a kernel gave up (1 s); the
+                                             launch is incomplete (see "State of W after a
+                                             timeout" below) */
 
 /* ---- switch kernel variants (adafuse_set_switch_kernel) ------------------ */
 #define ADAFUSE_KERNEL_AUTO      0  /* rank <= 8: TCGEN05; other multiples of 8: TCGEN05_PAIR;
@@ -237,6 +238,17 @@ ADAFUSE_API int adafuse_get_topk_switch_kernel(adafuse_ctx* ctx);
  * INVALID_ARG for any other value.  Host-only, no device work. */
 ADAFUSE_API int adafuse_set_tile_schedule(adafuse_ctx* ctx, int schedule);
 
+/* Cap the persistent grid of this context's switch and re-base launches at
+ * max_ctas CTAs (0 = no cap: one CTA per SM, two for the mma.sync kernel;
+ * the pair kernel rounds the cap down to whole CTA pairs, at least one).  A
+ * launch fills every SM it is given, so work on other streams cannot start
+ * beside it; a caller that pipelines the switch against its forward pass
+ * (adafuse_switch_batch_layers on a second stream) leaves SMs to the forward
+ * this way.  The grid only decides which CTA takes a tile, never how a tile
+ * is computed: W is bit for bit the same.  INVALID_ARG for max_ctas < 0.
+ * Host-only, no device work. */
+ADAFUSE_API int adafuse_set_max_ctas(adafuse_ctx* ctx, int32_t max_ctas);
+
 /* The kernel adafuse_switch will launch (ADAFUSE_KERNEL_MMA_SYNC,
  * ADAFUSE_KERNEL_TCGEN05, ADAFUSE_KERNEL_TCGEN05_PAIR or
  * ADAFUSE_KERNEL_TCGEN05_FOLD), or a negative code. */
@@ -282,6 +294,33 @@ ADAFUSE_API int adafuse_pregate_topk(adafuse_ctx* ctx, const float* h, int64_t T
                                      const float* Wr, int32_t k, adafuse_route4* route,
                                      void* stream);
 
+/* ---- batch decode ---------------------------------------------------------
+ * The pages make one routing decision per token (gist.science technical
+ * summary, section 2-ga).  A decode batch of T sequences that shares one
+ * merged weight can carry only one expert set, so these calls make ONE
+ * decision for the batch (a reading beyond the pages): the token rule applied
+ * to the mean of the batch's router logits,
+ *   zbar_e = (sum_t z_t,e) / T,  z_t,e as adafuse_pregate computes them,
+ * summed in token order in fp32; then the experts first under (zbar
+ * descending, index ascending) and gates = the softmax over all E of zbar
+ * renormalised over the picks.  With T = 1 the record equals the token's
+ * adafuse_pregate / adafuse_pregate_topk record bit for bit.  The result is
+ * one route record; pass it to adafuse_switch / adafuse_switch_topk like a
+ * token's route.
+ * Arguments as for adafuse_pregate; 1 <= T <= ADAFUSE_MAX_BATCH_TOKENS
+ * (INVALID_ARG above it; T == 0 is a no-op).  Two launches on `stream`: the
+ * tokens' logits into a context-owned scratch of ADAFUSE_MAX_BATCH_TOKENS x E
+ * fp32 (allocated at create), then the mean and the decision.  The scratch
+ * is shared by the context's calls; calls on one stream are ordered. */
+#define ADAFUSE_MAX_BATCH_TOKENS 4096
+ADAFUSE_API int adafuse_pregate_batch(adafuse_ctx* ctx, const float* h, int64_t T, int64_t d,
+                                      const float* Wr, adafuse_route* route, void* stream);
+
+/* As adafuse_pregate_batch with k in [1, 4] picks into one adafuse_route4. */
+ADAFUSE_API int adafuse_pregate_batch_topk(adafuse_ctx* ctx, const float* h, int64_t T,
+                                           int64_t d, const float* Wr, int32_t k,
+                                           adafuse_route4* route, void* stream);
+
 /* As adafuse_switch with top-k routes: per expert e in prev U cur the
  * coefficient is c_e = s*(g_cur(e) - g_prev(e)), experts with c_e == 0 are
  * dropped, and W <- bf16_rne(W + sum_e c_e B_e A_e) with fp32 accumulation
@@ -307,14 +346,38 @@ ADAFUSE_API int adafuse_rebase_topk(adafuse_ctx* ctx, const adafuse_route4* cur,
  * of the B tensors in device memory. */
 ADAFUSE_API int adafuse_refresh_adapters(adafuse_ctx* ctx, void* stream);
 
+/* State of W after a timeout.  The tensor-core kernels bound every wait;
+ * when one runs out the launch raises ADAFUSE_STATUS_TIMEOUT and its CTAs stop
+ * where they are.  Each 128 x 128 tile of the segment table is updated in
+ * shared memory as a whole and written back by one store, after its whole
+ * update, so after the stop every tile is in one of two states: switched
+ * (its new values were stored before the stop) or untouched (it keeps its
+ * values from before the launch).  No tile is partly switched, but which
+ * tiles were reached is not recorded.  An in-place switch is not idempotent:
+ * running the same switch again would apply it twice to the switched tiles.
+ * Recovery: with a pristine copy registered (adafuse_set_base),
+ * adafuse_rebase(ctx, cur) rewrites every tile as bf16_rne(W0 + s * sum_{e in
+ * cur} g_e B_e A_e), a consistent state for the route `cur`; without one, the
+ * caller restores W from its own copy of the weights.  A re-base that timed
+ * out is recovered by running it again.  The mma.sync kernel has no waits
+ * and never times out. */
+
 /* Test hook for the timeout path (no counterpart on the pages).  The next
  * switch or re-base launched with a tensor-core kernel announces 16 bytes of
- * operand transfers that never arrive on each CTA's first stage, so the MMA
- * warp's bounded wait (1 s) runs out: the launch raises
- * ADAFUSE_STATUS_TIMEOUT, every warp leaves through its bounded waits, TMEM is
- * freed, no MMA completes and W is not written; the context stays usable.
- * UNSUPPORTED_SHAPE when the context's kernel is ADAFUSE_KERNEL_MMA_SYNC (it
- * has no waits).  Host-only; consumed by the next launch. */
+ * operand transfers that never arrive on the first operand stage of the
+ * `tile`-th tile (1-based) that each CTA -- each CTA pair for
+ * ADAFUSE_KERNEL_TCGEN05_PAIR -- takes, so the MMA warp's bounded wait (1 s)
+ * runs out: the launch raises ADAFUSE_STATUS_TIMEOUT, every warp leaves
+ * through its bounded waits and TMEM is freed; the context stays usable.  A
+ * CTA's tiles before that one are switched and stored, that tile and later
+ * ones are untouched (the state described above); with tile == 1 nothing is
+ * written.  INVALID_ARG when tile < 1; UNSUPPORTED_SHAPE when the context's
+ * kernel is ADAFUSE_KERNEL_MMA_SYNC (it has no waits).  Host-only; consumed
+ * by the next launch. */
+ADAFUSE_API int adafuse_debug_stall_next_switch_at(adafuse_ctx* ctx, int32_t tile);
+
+/* adafuse_debug_stall_next_switch_at(ctx, 1): the next launch stalls on each
+ * CTA's first tile and writes no W. */
 ADAFUSE_API int adafuse_debug_stall_next_switch(adafuse_ctx* ctx);
 
 /* Synchronise `stream`, read the device status word into *status, then

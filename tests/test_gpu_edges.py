@@ -203,6 +203,71 @@ def test_bounded_wait_timeout_reports_status_and_context_stays_usable(kernel, r)
     _switch_and_check(cfg, m, sw, routes, [(None, 0), (0, 1)])
 
 
+@pytest.mark.parametrize("kernel,r", [(TC, 8), (TC2, 16), (TF, 8), (TC, 32)])
+def test_timeout_mid_launch_leaves_whole_tiles_and_rebase_recovers(kernel, r):
+    """A bounded wait that runs out in the middle of a switch: the hook
+    stalls each CTA's second tile, so every CTA stores its first tile and
+    stops.  Every 128 x 128 tile must then be either untouched or fully
+    switched (the oracle's prev -> cur result), with both kinds present; the
+    documented recovery, a re-base from the registered pristine weights,
+    gives the oracle's W0 + dW(cur) everywhere."""
+    cfg = wl.custom("mid", 2, [("q", 1024, 1024), ("o", 1280, 768)], n_experts=4, rank=r,
+                    alpha=2.0 * r, n_tokens=2, d=1024)
+    m = wl.make_model(cfg, device="cuda", seed=90 + r)
+    sw = Bnd.Switcher(m.W, m.A, m.B, cfg.n_layers, len(cfg.targets), cfg.n_experts, cfg.rank,
+                      cfg.alpha, device=torch.cuda.current_device())
+    sw.set_kernel(kernel)
+    base = [w.clone() for w in m.W]
+    sw.set_base(base)
+    W0 = [bits(w) for w in base]
+    A_h, B_h = [bits(a) for a in m.A], [bits(b) for b in m.B]
+    routes = make_routes(np.array([[0, 2], [3, 1]], np.int32),
+                         np.array([[0.7, 0.3], [0.6, 0.4]], np.float32))
+    r_np = routes_to_np(routes)
+    p = lambda t: Bnd.Switcher.route_ptr(routes, t)
+    sw.switch(None, p(0), stream())
+    torch.cuda.synchronize()
+    assert sw.status(stream()) == 0
+    before = [bits(w) for w in m.W]
+    Bnd.adafuse_debug_stall_next_switch_at(sw.ctx, 2)
+    sw.switch(p(0), p(1), stream())
+    assert sw.status(stream()) == Bnd.ADAFUSE_STATUS_TIMEOUT
+    n_old = n_new = 0
+    for i, w in enumerate(m.W):
+        got = bits(w)
+        out, inn = got.shape
+        rows = np.arange(out, dtype=np.int64)
+        want, _ = oracle.switch_rows(before[i], rows, out, A_h[i], B_h[i], cfg.scale,
+                                     route_tuple(r_np, 0), route_tuple(r_np, 1), exact=True)
+        patched = got.copy()
+        for r0 in range(0, out, 128):
+            for c0 in range(0, inn, 128):
+                t_got = got[r0:r0 + 128, c0:c0 + 128]
+                if np.array_equal(t_got, before[i][r0:r0 + 128, c0:c0 + 128]):
+                    n_old += 1
+                    patched[r0:r0 + 128, c0:c0 + 128] = want[r0:r0 + 128, c0:c0 + 128]
+                else:
+                    n_new += 1
+        # every tile that changed holds the full prev -> cur switch
+        check_switch_rows(patched, before[i], rows, out, A_h[i], B_h[i], cfg.scale,
+                          route_tuple(r_np, 0), route_tuple(r_np, 1))
+    assert n_old > 0 and n_new > 0, (n_old, n_new)
+    # recovery: re-base every tile from the pristine weights onto route 1
+    sw.rebase(p(1), stream())
+    torch.cuda.synchronize()
+    assert sw.status(stream()) == 0
+    for i, w in enumerate(m.W):
+        rows = np.arange(w.shape[0], dtype=np.int64)
+        check_switch_rows(bits(w), W0[i], rows, w.shape[0], A_h[i], B_h[i], cfg.scale, None,
+                          route_tuple(r_np, 1))
+
+
+def test_stall_hook_rejects_a_tile_number_below_one():
+    cfg, m, sw = _model(TC, seed=23, r=8)
+    with pytest.raises(Bnd.AdafuseError):
+        Bnd.adafuse_debug_stall_next_switch_at(sw.ctx, 0)
+
+
 def test_stall_hook_is_refused_by_the_wait_free_kernel():
     cfg, m, sw = _model(MMA, seed=22, r=8)
     with pytest.raises(Bnd.AdafuseError):

@@ -325,6 +325,34 @@ def test_pipelined_switch_against_a_forward_equals_one_full_switch(kernel, r):
         torch.testing.assert_close(y, torch.mv(m1.W[i], xs[i % nt]), rtol=0, atol=0)
 
 
+@pytest.mark.parametrize("kernel,r,cap", [(TC, 8, 7), (TC, 16, 1), (TC2, 16, 7), (TC2, 64, 2),
+                                           (TF, 8, 5), (MMA, 12, 3)])
+def test_grid_cap_gives_the_same_w_bit_for_bit(kernel, r, cap):
+    """adafuse_set_max_ctas only shrinks the persistent grid: each tile is
+    computed the same way whichever CTA takes it, so a capped context and an
+    uncapped one end with the same W, bit for bit, over full and layer-range
+    switches (both tile schedules of the single-CTA kernel)."""
+    m1, m2 = _small_model(seed=23, r=r), _small_model(seed=23, r=r)
+    s1, s2 = make_switcher(m1, kernel), make_switcher(m2, kernel)
+    s2.set_max_ctas(cap)
+    if kernel == TC:
+        s1.set_schedule(Bnd.ADAFUSE_SCHEDULE_STATIC)
+    routes = make_routes(np.array([[0, 1], [2, 3], [1, 2]], np.int32),
+                         np.array([[0.7, 0.3], [0.6, 0.4], [0.5, 0.5]], np.float32))
+    p = lambda t: Bnd.Switcher.route_ptr(routes, t)
+    for sw in (s1, s2):
+        sw.switch(None, p(0), stream())
+        sw.switch(p(0), p(1), stream())
+        sw.switch_layers(1, 2, p(1), p(2), stream())
+        sw.switch_layers(0, 1, p(1), p(2), stream())
+    torch.cuda.synchronize()
+    assert s1.status(stream()) == 0 and s2.status(stream()) == 0
+    for a, b in zip(m1.W, m2.W):
+        assert np.array_equal(bits(a), bits(b))
+    with pytest.raises(Bnd.AdafuseError):
+        s2.set_max_ctas(-1)
+
+
 @pytest.mark.parametrize("r", [8, 4, 16])
 def test_static_and_dynamic_tile_schedules_agree_bitwise(r):
     """The schedule only decides which CTA takes a tile, never how a tile is

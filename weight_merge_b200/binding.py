@@ -32,6 +32,7 @@ ADAFUSE_KERNEL_TCGEN05_FOLD = 4
 ADAFUSE_SCHEDULE_STATIC = 0
 ADAFUSE_SCHEDULE_DYNAMIC = 1
 ADAFUSE_MAX_TOP_K = 4
+ADAFUSE_MAX_BATCH_TOKENS = 4096
 
 
 class AdafuseError(RuntimeError):
@@ -90,16 +91,20 @@ def lib() -> ctypes.CDLL:
         "adafuse_get_device_status": ([P, P, ctypes.POINTER(i32)], ctypes.c_int),
         "adafuse_set_switch_kernel": ([P, ctypes.c_int], ctypes.c_int),
         "adafuse_set_tile_schedule": ([P, ctypes.c_int], ctypes.c_int),
+        "adafuse_set_max_ctas": ([P, i32], ctypes.c_int),
         "adafuse_get_topk_switch_kernel": ([P], ctypes.c_int),
         "adafuse_set_base": ([P, ctypes.POINTER(P)], ctypes.c_int),
         "adafuse_rebase": ([P, P, P], ctypes.c_int),
         "adafuse_rebase_layers": ([P, i32, i32, P, P], ctypes.c_int),
         "adafuse_get_switch_kernel": ([P], ctypes.c_int),
         "adafuse_pregate_topk": ([P, P, i64, i64, P, i32, P, P], ctypes.c_int),
+        "adafuse_pregate_batch": ([P, P, i64, i64, P, P, P], ctypes.c_int),
+        "adafuse_pregate_batch_topk": ([P, P, i64, i64, P, i32, P, P], ctypes.c_int),
         "adafuse_switch_topk": ([P, P, P, P], ctypes.c_int),
         "adafuse_switch_topk_layers": ([P, i32, i32, P, P, P], ctypes.c_int),
         "adafuse_rebase_topk": ([P, P, P], ctypes.c_int),
         "adafuse_debug_stall_next_switch": ([P], ctypes.c_int),
+        "adafuse_debug_stall_next_switch_at": ([P, i32], ctypes.c_int),
         "adafuse_refresh_adapters": ([P, P], ctypes.c_int),
         "adafuse_segment_table": ([ctypes.POINTER(Desc), P, i64, ctypes.POINTER(i64)], ctypes.c_int),
         "adafuse_tile_size": ([], ctypes.c_int),
@@ -181,6 +186,18 @@ def adafuse_pregate_topk(ctx: int, h: int, T: int, d: int, Wr: int, k: int, rout
            "adafuse_pregate_topk")
 
 
+def adafuse_pregate_batch(ctx: int, h: int, T: int, d: int, Wr: int, route: int,
+                          stream: int = 0) -> None:
+    _check(lib().adafuse_pregate_batch(ctx, h, int(T), int(d), Wr, route, stream or None),
+           "adafuse_pregate_batch")
+
+
+def adafuse_pregate_batch_topk(ctx: int, h: int, T: int, d: int, Wr: int, k: int, route: int,
+                               stream: int = 0) -> None:
+    _check(lib().adafuse_pregate_batch_topk(ctx, h, int(T), int(d), Wr, int(k), route,
+                                            stream or None), "adafuse_pregate_batch_topk")
+
+
 def adafuse_switch_topk(ctx: int, prev: Optional[int], cur: Optional[int], stream: int = 0) -> None:
     _check(lib().adafuse_switch_topk(ctx, prev or None, cur or None, stream or None),
            "adafuse_switch_topk")
@@ -205,12 +222,21 @@ def adafuse_debug_stall_next_switch(ctx: int) -> None:
     _check(lib().adafuse_debug_stall_next_switch(ctx), "adafuse_debug_stall_next_switch")
 
 
+def adafuse_debug_stall_next_switch_at(ctx: int, tile: int) -> None:
+    _check(lib().adafuse_debug_stall_next_switch_at(ctx, int(tile)),
+           "adafuse_debug_stall_next_switch_at")
+
+
 def adafuse_set_switch_kernel(ctx: int, kernel: int) -> None:
     _check(lib().adafuse_set_switch_kernel(ctx, int(kernel)), "adafuse_set_switch_kernel")
 
 
 def adafuse_set_tile_schedule(ctx: int, schedule: int) -> None:
     _check(lib().adafuse_set_tile_schedule(ctx, int(schedule)), "adafuse_set_tile_schedule")
+
+
+def adafuse_set_max_ctas(ctx: int, max_ctas: int) -> None:
+    _check(lib().adafuse_set_max_ctas(ctx, int(max_ctas)), "adafuse_set_max_ctas")
 
 
 def adafuse_get_topk_switch_kernel(ctx: int) -> int:
@@ -328,6 +354,17 @@ class Switcher:
         adafuse_pregate_topk(self.ctx, h.data_ptr(), T, d, Wr.data_ptr(), k, routes.data_ptr(),
                              stream)
 
+    def pregate_batch(self, h, Wr, route, stream: int = 0) -> None:
+        """One top-2 route for the whole batch h [T, d] into ``route`` (one
+        16-byte record, e.g. a row of an int32 [n, 4] buffer)."""
+        T, d = h.shape
+        adafuse_pregate_batch(self.ctx, h.data_ptr(), T, d, Wr.data_ptr(), route.data_ptr(), stream)
+
+    def pregate_batch_topk(self, h, Wr, k: int, route, stream: int = 0) -> None:
+        T, d = h.shape
+        adafuse_pregate_batch_topk(self.ctx, h.data_ptr(), T, d, Wr.data_ptr(), k,
+                                   route.data_ptr(), stream)
+
     def switch_topk(self, prev: Optional[int], cur: Optional[int], stream: int = 0) -> None:
         adafuse_switch_topk(self.ctx, prev, cur, stream)
 
@@ -343,6 +380,9 @@ class Switcher:
 
     def set_schedule(self, schedule: int) -> None:
         adafuse_set_tile_schedule(self.ctx, schedule)
+
+    def set_max_ctas(self, max_ctas: int) -> None:
+        adafuse_set_max_ctas(self.ctx, max_ctas)
 
     @property
     def kernel(self) -> int:

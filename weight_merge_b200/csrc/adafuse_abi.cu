@@ -8,6 +8,7 @@
 #include <cstdio>
 #include <cstring>
 #include <algorithm>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -36,17 +37,19 @@ struct adafuse_ctx {
     std::vector<PairDesc> h_pairs;  // host copy of d_pairs (re-base pointers are patched in)
     CUtensorMap* d_w0_maps = nullptr;  // 1 per pair on the re-base source W0
     bool has_base = false;
-    bool stall_next = false;  // test hook: the next tensor-core launch times out
+    int stall_at = 0;  // test hook: the next tensor-core launch stalls at each CTA's n-th tile
     // pair kernel: 256 x 128 blocks, layer-major like the tile table
     TileEntry* d_blocks = nullptr;
     uint16_t* d_bpad = nullptr;              // rank < 8: B with rows zero-padded to 8
     uint16_t* d_fold = nullptr;              // rank <= 8: folded-coefficient operands
                                              // (allocated on first use, see ensure_fold)
     bool fold_failed = false;                // that allocation failed: the kernel is off
+    float* d_logits = nullptr;               // [kMaxBatchTokens, E] batch pre-gate scratch
     unsigned long long* d_sched = nullptr;   // [2] ticket counter of the dynamic tile schedule
     int schedule = ADAFUSE_SCHEDULE_DYNAMIC;
     std::vector<int64_t> layer_block_begin;  // [n_layers + 1]
     int pair_clusters = 0;                   // co-resident CTA pairs (0 = not queried yet)
+    int max_ctas = 0;                        // cap on a switch's persistent grid (0 = none)
 };
 
 namespace {
@@ -73,7 +76,42 @@ struct DeviceGuard {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// CTAs a switch launch may keep resident: every SM, or the caller's cap
+// (adafuse_set_max_ctas) so that other work can run beside the switch.
+int switch_ctas(const adafuse_ctx* c) {
+    return c->max_ctas > 0 && c->max_ctas < c->sm_count ? c->max_ctas : c->sm_count;
+}
+
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Raise a kernel's dynamic shared-memory limit only when this device has not
+// been given at least `bytes` for that kernel yet (the host call is not free,
+// and the decode-time pre-gate launches are short).  Keyed by the kernel's
+// address and the device: kernels of one signature are different entries.
+struct SmemAttrEntry {
+    const void* fn;
+    int device;
+    size_t bytes;
+};
+
+template <typename Kernel>
+void ensure_smem_attr(Kernel kernel, size_t bytes, int device) {
+    static std::mutex mu;
+    static std::vector<SmemAttrEntry> done;
+    const void* fn = reinterpret_cast<const void*>(kernel);
+    std::lock_guard<std::mutex> lk(mu);
+    for (const SmemAttrEntry& en : done)
+        if (en.fn == fn && en.device == device && en.bytes >= bytes) return;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
+        cudaSuccess)
+        return;   // the launch reports the error
+    for (SmemAttrEntry& en : done)
+        if (en.fn == fn && en.device == device) {
+            en.bytes = bytes;
+            return;
+        }
+    done.push_back({fn, device, bytes});
+}
 
 // Shape and pointer checks shared by create and the host-only table query.
 int check_desc(const adafuse_desc* d, bool need_pointers) {
@@ -223,11 +261,11 @@ cudaError_t launch_tc(adafuse_ctx* c, int64_t t0, int64_t t1, const int32_t* pre
     prm.status = c->d_status;
     prm.rebase = rebase ? 1 : 0;
     prm.w0_maps = c->d_w0_maps;
-    prm.stall = c->stall_next ? 1 : 0;
-    c->stall_next = false;
+    prm.stall = c->stall_at;
+    c->stall_at = 0;
     prm.dyn = c->schedule == ADAFUSE_SCHEDULE_DYNAMIC ? 1 : 0;
     prm.sched = c->d_sched;
-    return launch_switch_tc<KP, BBULK>(prm, c->device, c->sm_count, s);
+    return launch_switch_tc<KP, BBULK>(prm, c->device, switch_ctas(c), s);
 }
 
 template <int KP>
@@ -254,11 +292,12 @@ cudaError_t launch_tc2(adafuse_ctx* c, int64_t b0, int64_t b1, const int32_t* pr
     prm.status = c->d_status;
     prm.rebase = rebase ? 1 : 0;
     prm.w0_maps = c->d_w0_maps;
-    prm.stall = c->stall_next ? 1 : 0;
-    c->stall_next = false;
+    prm.stall = c->stall_at;
+    c->stall_at = 0;
     prm.dyn = 0;
     prm.sched = nullptr;
-    return launch_switch_tc2<KP>(prm, c->pair_clusters, s);
+    const int cap = switch_ctas(c) / 2 > 0 ? switch_ctas(c) / 2 : 1;
+    return launch_switch_tc2<KP>(prm, c->pair_clusters < cap ? c->pair_clusters : cap, s);
 }
 
 }  // namespace
@@ -377,6 +416,7 @@ int adafuse_create(adafuse_ctx** out, const adafuse_desc* desc, int device) {
         cudaFree(c->d_bpad);
         cudaFree(c->d_fold);
         cudaFree(c->d_sched);
+        cudaFree(c->d_logits);
         delete c;
         return err == cudaErrorMemoryAllocation ? ADAFUSE_ERR_OUT_OF_MEMORY : cuda_fail(err, what);
     };
@@ -404,6 +444,8 @@ int adafuse_create(adafuse_ctx** out, const adafuse_desc* desc, int device) {
         return fail(e, "cudaMalloc(tiles)");
     if ((e = cudaMalloc(&c->d_status, sizeof(int32_t))) != cudaSuccess)
         return fail(e, "cudaMalloc(status)");
+    if ((e = cudaMalloc(&c->d_logits, sizeof(float) * kMaxBatchTokens * desc->n_experts)) != cudaSuccess)
+        return fail(e, "cudaMalloc(batch logits)");
     if ((e = cudaMalloc(&c->d_sched, 2 * sizeof(unsigned long long))) != cudaSuccess)
         return fail(e, "cudaMalloc(schedule)");
     if ((e = cudaMemset(c->d_sched, 0, 2 * sizeof(unsigned long long))) != cudaSuccess)
@@ -482,6 +524,7 @@ int adafuse_destroy(adafuse_ctx* ctx) {
     cudaFree(ctx->d_bpad);
     cudaFree(ctx->d_fold);
     cudaFree(ctx->d_sched);
+    cudaFree(ctx->d_logits);
     delete ctx;
     return ADAFUSE_OK;
 }
@@ -523,6 +566,12 @@ int adafuse_set_tile_schedule(adafuse_ctx* ctx, int schedule) {
     return ADAFUSE_OK;
 }
 
+int adafuse_set_max_ctas(adafuse_ctx* ctx, int32_t max_ctas) {
+    if (ctx == nullptr || max_ctas < 0) return ADAFUSE_ERR_INVALID_ARG;
+    ctx->max_ctas = max_ctas;
+    return ADAFUSE_OK;
+}
+
 int adafuse_get_switch_kernel(adafuse_ctx* ctx) {
     if (ctx == nullptr) return ADAFUSE_ERR_INVALID_ARG;
     if (ctx->kernel == ADAFUSE_KERNEL_AUTO) {
@@ -542,28 +591,54 @@ namespace {
 // Top-k pre-gating into routes of `slots` slots (2: adafuse_route, 4:
 // adafuse_route4).  The same kernels and arithmetic for every k and batch.
 int pregate_launch(adafuse_ctx* ctx, const float* h, int64_t T, int64_t d, const float* Wr,
-                   int k, int slots, void* route_out, void* stream) {
+                   int k, int slots, void* route_out, void* stream, float* logits = nullptr) {
     int32_t* route = static_cast<int32_t*>(route_out);
     if (ctx == nullptr || T < 0 || d < 1 || (d & 3) != 0) return ADAFUSE_ERR_INVALID_ARG;
     if (T == 0) return ADAFUSE_OK;
-    if (h == nullptr || Wr == nullptr || route == nullptr) return ADAFUSE_ERR_INVALID_ARG;
+    if (h == nullptr || Wr == nullptr || (route == nullptr && logits == nullptr))
+        return ADAFUSE_ERR_INVALID_ARG;
     if (!aligned16(h) || !aligned16(route) || (reinterpret_cast<uintptr_t>(Wr) & 3u))
         return ADAFUSE_ERR_INVALID_ARG;
     DeviceGuard guard(ctx->device);
     if (!guard.ok) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int E = ctx->n_experts;
+    // Batches of 64+ tokens with up to 8 experts and d <= 4096: the
+    // token-group kernel (one warp per 4 tokens).  It computes the same bits
+    // as pregate_kernel, which takes every other case, so a token's route
+    // does not depend on which one ran.
+    const int64_t nch = ceil_div(d >> 2, 256);
+    if (E <= 8 && nch <= kGroupMaxChunks && T >= kGroupMinTokens) {
+        const size_t smem = group_smem_bytes(d);
+        const int64_t ngroups = ceil_div(T, kGroupTokens);
+        const unsigned grid = (unsigned)std::min<int64_t>(ngroups, (int64_t)ctx->sm_count);
+        auto go = [&](auto kernel) {
+            ensure_smem_attr(kernel, smem, ctx->device);
+            kernel<<<grid, kGroupThreads, smem, s>>>(h, T, d, Wr, E, k, slots, route, logits);
+        };
+        switch (nch) {
+            case 1: go(pregate_group_kernel<1>); break;
+            case 2: go(pregate_group_kernel<2>); break;
+            case 3: go(pregate_group_kernel<3>); break;
+            default: go(pregate_group_kernel<4>); break;
+        }
+        const cudaError_t e = cudaGetLastError();
+        return e == cudaSuccess ? ADAFUSE_OK : cuda_fail(e, "pregate launch");
+    }
     const int emax = E <= 8 ? 8 : E <= 16 ? 16 : E <= 32 ? 32 : 64;
     const int tpb = 64 / emax;   // tokens per CTA group: TPB x EMAX partial logits per thread
     const int64_t groups = ceil_div(T, tpb);
     // Wr in shared memory for batches that amortise staging it (persistent
     // CTAs); otherwise read from global memory.  Same arithmetic either way.
+    // Rows of Wr are read as float4 only when Wr is 16-byte aligned (the ABI
+    // asks for 4-byte alignment); otherwise element by element.
+    const bool wr16 = (reinterpret_cast<uintptr_t>(Wr) & 15u) == 0;
     const size_t wr_smem = (size_t)d * (emax + 1) * 4;
     const bool shared = T >= 256 && wr_smem <= 160 * 1024;
     const unsigned grid = (unsigned)(shared ? std::min<int64_t>(groups, (int64_t)ctx->sm_count) : groups);
     auto go = [&](auto kernel, size_t smem) {
-        if (smem > 0) cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        kernel<<<grid, kPregateThreads, smem, s>>>(h, T, d, Wr, E, k, slots, route);
+        if (smem > 0) ensure_smem_attr(kernel, smem, ctx->device);
+        kernel<<<grid, kPregateThreads, smem, s>>>(h, T, d, Wr, E, k, slots, route, logits);
     };
     if (shared) {
         switch (emax) {
@@ -572,7 +647,7 @@ int pregate_launch(adafuse_ctx* ctx, const float* h, int64_t T, int64_t d, const
             case 32: go(pregate_kernel<32, 2, kWrShared>, wr_smem); break;
             default: go(pregate_kernel<64, 1, kWrShared>, wr_smem); break;
         }
-    } else if (E == emax) {
+    } else if (E == emax && wr16) {
         switch (emax) {
             case 8: go(pregate_kernel<8, 8, kWrVector>, 0); break;
             case 16: go(pregate_kernel<16, 4, kWrVector>, 0); break;
@@ -604,6 +679,51 @@ int adafuse_pregate_topk(adafuse_ctx* ctx, const float* h, int64_t T, int64_t d,
                          const float* Wr, int32_t k, adafuse_route4* route, void* stream) {
     if (k < 1 || k > ADAFUSE_MAX_TOP_K) return ADAFUSE_ERR_INVALID_ARG;
     return pregate_launch(ctx, h, T, d, Wr, k, 4, route, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+// One routing decision for the whole batch: the tokens' logits into the
+// context's scratch (the per-token kernels, same arithmetic), then their
+// mean and the token rule in one more launch.
+int pregate_batch_launch(adafuse_ctx* ctx, const float* h, int64_t T, int64_t d, const float* Wr,
+                         int k, int slots, void* route_out, void* stream) {
+    if (ctx == nullptr || T < 0 || T > kMaxBatchTokens) return ADAFUSE_ERR_INVALID_ARG;
+    if (T == 0) return ADAFUSE_OK;
+    if (route_out == nullptr || !aligned16(route_out)) return ADAFUSE_ERR_INVALID_ARG;
+    const int rc = pregate_launch(ctx, h, T, d, Wr, k, slots, nullptr, stream, ctx->d_logits);
+    if (rc != ADAFUSE_OK) return rc;
+    DeviceGuard guard(ctx->device);
+    if (!guard.ok) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t* route = static_cast<int32_t*>(route_out);
+    const int E = ctx->n_experts;
+    switch (E <= 8 ? 8 : E <= 16 ? 16 : E <= 32 ? 32 : 64) {
+        case 8: pregate_batch_reduce_kernel<8><<<1, 64, 0, s>>>(ctx->d_logits, T, E, k, slots, route); break;
+        case 16: pregate_batch_reduce_kernel<16><<<1, 64, 0, s>>>(ctx->d_logits, T, E, k, slots, route); break;
+        case 32: pregate_batch_reduce_kernel<32><<<1, 64, 0, s>>>(ctx->d_logits, T, E, k, slots, route); break;
+        default: pregate_batch_reduce_kernel<64><<<1, 64, 0, s>>>(ctx->d_logits, T, E, k, slots, route); break;
+    }
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? ADAFUSE_OK : cuda_fail(e, "batch pregate launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+int adafuse_pregate_batch(adafuse_ctx* ctx, const float* h, int64_t T, int64_t d,
+                          const float* Wr, adafuse_route* route, void* stream) {
+    return pregate_batch_launch(ctx, h, T, d, Wr, 2, 2, route, stream);
+}
+
+int adafuse_pregate_batch_topk(adafuse_ctx* ctx, const float* h, int64_t T, int64_t d,
+                               const float* Wr, int32_t k, adafuse_route4* route,
+                               void* stream) {
+    if (k < 1 || k > ADAFUSE_MAX_TOP_K) return ADAFUSE_ERR_INVALID_ARG;
+    return pregate_batch_launch(ctx, h, T, d, Wr, k, 4, route, stream);
 }
 
 }  // extern "C"
@@ -664,14 +784,14 @@ int launch_switch(adafuse_ctx* ctx, int32_t layer_begin, int32_t n_layers,
         prm.status = ctx->d_status;
         prm.rebase = rebase ? 1 : 0;
         prm.w0_maps = ctx->d_w0_maps;
-        prm.stall = ctx->stall_next ? 1 : 0;
-        ctx->stall_next = false;
+        prm.stall = ctx->stall_at;
+        ctx->stall_at = 0;
         prm.dyn = 0;
         prm.sched = nullptr;
         const int64_t w0 = (int64_t)layer_begin * ctx->n_targets;
         const int64_t nw = (int64_t)n_layers * ctx->n_targets;
         const cudaError_t e =
-            launch_switch_fold(prm, w0, nw, ctx->rank, ctx->device, ctx->sm_count, s);
+            launch_switch_fold(prm, w0, nw, ctx->rank, ctx->device, switch_ctas(ctx), s);
         return e == cudaSuccess ? ADAFUSE_OK : cuda_fail(e, "switch launch");
     }
     if (kind == ADAFUSE_KERNEL_TCGEN05) {
@@ -686,7 +806,7 @@ int launch_switch(adafuse_ctx* ctx, int32_t layer_begin, int32_t n_layers,
             e = launch_tc<64, false>(ctx, t0, t1, prev, cur, slots, s, rebase);
         return e == cudaSuccess ? ADAFUSE_OK : cuda_fail(e, "switch launch");
     }
-    const int64_t want = (int64_t)ctx->sm_count * 2;
+    const int64_t want = (int64_t)switch_ctas(ctx) * 2;
     const unsigned grid = (unsigned)(t1 - t0 < want ? t1 - t0 : want);
     const int E = ctx->n_experts, r = ctx->rank;
     const float sc = ctx->scale;
@@ -808,11 +928,15 @@ int adafuse_refresh_adapters(adafuse_ctx* ctx, void* stream) {
     return e == cudaSuccess ? ADAFUSE_OK : cuda_fail(e, "cudaMemcpy2D(padded B)");
 }
 
-int adafuse_debug_stall_next_switch(adafuse_ctx* ctx) {
-    if (ctx == nullptr) return ADAFUSE_ERR_INVALID_ARG;
+int adafuse_debug_stall_next_switch_at(adafuse_ctx* ctx, int32_t tile) {
+    if (ctx == nullptr || tile < 1) return ADAFUSE_ERR_INVALID_ARG;
     if (adafuse_get_switch_kernel(ctx) == ADAFUSE_KERNEL_MMA_SYNC) return ADAFUSE_ERR_UNSUPPORTED_SHAPE;
-    ctx->stall_next = true;
+    ctx->stall_at = tile;
     return ADAFUSE_OK;
+}
+
+int adafuse_debug_stall_next_switch(adafuse_ctx* ctx) {
+    return adafuse_debug_stall_next_switch_at(ctx, 1);
 }
 
 int adafuse_get_device_status(adafuse_ctx* ctx, void* stream, int32_t* status) {

@@ -23,16 +23,66 @@
 #pragma once
 
 #include "common.cuh"
+#include "sm100_ptx.cuh"
 
 namespace adafuse {
 
 constexpr int kPregateThreads = 256;
 enum : int { kWrShared = 0, kWrVector = 1, kWrScalar = 2 };
 
+// The routing decision of one token from its logits z[0..E): top-k under
+// (z descending, index ascending) -- pick j is the largest logit not yet
+// picked, the lower index among equals -- and gates = the softmax over all E
+// renormalised over the picks, in the closed form g_j = x_j / (1 + x_1 +
+// ...), x_j = exp(z_j - z_0) <= 1.  Written as one adafuse_route (slots 2) or
+// adafuse_route4 (slots 4) record at index t.
+template <int EMAX>
+__device__ __forceinline__ void route_tail(const float (&z)[EMAX], int E, int k, int slots,
+                                           int32_t* __restrict__ route, int64_t t) {
+    int pick[4] = {-1, -1, -1, -1};
+    float zp[4] = {0.f, 0.f, 0.f, 0.f};
+    uint64_t taken = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        if (j >= k) break;
+        int best = -1;
+        float zb = 0.f;
+#pragma unroll
+        for (int e = 0; e < EMAX; ++e) {
+            if (e >= E || ((taken >> e) & 1ull)) continue;
+            if (best < 0 || z[e] > zb) { best = e; zb = z[e]; }
+        }
+        if (best < 0) break;
+        pick[j] = best;
+        zp[j] = zb;
+        taken |= 1ull << best;
+    }
+    float x[4] = {1.f, 0.f, 0.f, 0.f};
+    float den = 1.f;
+#pragma unroll
+    for (int j = 1; j < 4; ++j)
+        if (pick[j] >= 0) {
+            x[j] = expf(zp[j] - zp[0]);
+            den = den + x[j];
+        }
+    float g[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) g[j] = pick[j] >= 0 ? x[j] / den : 0.f;
+    if (slots == 2) {
+        reinterpret_cast<int4*>(route)[t] =
+            make_int4(pick[0], pick[1], __float_as_int(g[0]), __float_as_int(g[1]));
+    } else {
+        int4* r4 = reinterpret_cast<int4*>(route) + 2 * t;
+        r4[0] = make_int4(pick[0], pick[1], pick[2], pick[3]);
+        r4[1] = make_int4(__float_as_int(g[0]), __float_as_int(g[1]), __float_as_int(g[2]),
+                          __float_as_int(g[3]));
+    }
+}
+
 template <int EMAX, int TPB, int WR>
 __global__ void __launch_bounds__(kPregateThreads)
 pregate_kernel(const float* __restrict__ h, int64_t T, int64_t d, const float* __restrict__ Wr,
-               int E, int k, int slots, int32_t* __restrict__ route) {
+               int E, int k, int slots, int32_t* __restrict__ route, float* __restrict__ logits) {
     static_assert(EMAX % 4 == 0, "EMAX");
     constexpr int kWarps = kPregateThreads / 32;
     constexpr int S4 = EMAX + 1;             // float4 slots per chunk in shared memory
@@ -42,7 +92,7 @@ pregate_kernel(const float* __restrict__ h, int64_t T, int64_t d, const float* _
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if constexpr (WR == kWrShared) {
-        if (E == EMAX) {
+        if (E == EMAX && (reinterpret_cast<uintptr_t>(Wr) & 15u) == 0) {
             // a 4-row chunk of Wr is EMAX contiguous float4 in global memory
             const float4* src = reinterpret_cast<const float4*>(Wr);
 #pragma unroll 8
@@ -127,50 +177,221 @@ pregate_kernel(const float* __restrict__ h, int64_t T, int64_t d, const float* _
                 for (int w = 1; w < kWarps; ++w) v += part[w][tt][e];
                 z[e] = v;
             }
-            // top-k under (z descending, index ascending): pick j is the
-            // largest logit not yet picked, the lower index among equals
-            int pick[4] = {-1, -1, -1, -1};
-            float zp[4] = {0.f, 0.f, 0.f, 0.f};
-            uint64_t taken = 0;
+            if (logits != nullptr) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                if (j >= k) break;
-                int best = -1;
-                float zb = 0.f;
-#pragma unroll
-                for (int e = 0; e < EMAX; ++e) {
-                    if (e >= E || ((taken >> e) & 1ull)) continue;
-                    if (best < 0 || z[e] > zb) { best = e; zb = z[e]; }
-                }
-                if (best < 0) break;
-                pick[j] = best;
-                zp[j] = zb;
-                taken |= 1ull << best;
-            }
-            // softmax over all E renormalised over the picks == softmax of the
-            // picked logits: g_j = x_j / (1 + x_1 + ...), x_j = exp(z_j - z_0) <= 1
-            float x[4] = {1.f, 0.f, 0.f, 0.f};
-            float den = 1.f;
-#pragma unroll
-            for (int j = 1; j < 4; ++j)
-                if (pick[j] >= 0) {
-                    x[j] = expf(zp[j] - zp[0]);
-                    den = den + x[j];
-                }
-            float g[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) g[j] = pick[j] >= 0 ? x[j] / den : 0.f;
-            if (slots == 2) {
-                reinterpret_cast<int4*>(route)[t0 + tt] =
-                    make_int4(pick[0], pick[1], __float_as_int(g[0]), __float_as_int(g[1]));
+                for (int e = 0; e < EMAX; ++e)
+                    if (e < E) logits[(t0 + tt) * E + e] = z[e];
             } else {
-                int4* r4 = reinterpret_cast<int4*>(route) + 2 * (t0 + tt);
-                r4[0] = make_int4(pick[0], pick[1], pick[2], pick[3]);
-                r4[1] = make_int4(__float_as_int(g[0]), __float_as_int(g[1]), __float_as_int(g[2]),
-                                  __float_as_int(g[3]));
+                route_tail<EMAX>(z, E, k, slots, route, t0 + tt);
             }
         }
         __syncthreads();   // part[] is reused by the next token group
+    }
+}
+
+
+// ---------------------------------------------------------------------------
+// Token-group form of the same router for batches (E <= 8, d <= 4096).  It
+// computes every logit with exactly the operation sequence of pregate_kernel
+// above -- virtual thread i = 32 * vw + lane of a 256-thread group (vw = 0..7)
+// accumulates the float4 chunks i, i + 256, ... in order (one fp32 FMA per
+// element and expert), the xor tree at lane distances 16, 8, 4, 2, 1 finishes
+// each virtual warp's sum, and the eight virtual-warp sums are added in order
+// -- so both kernels give the same bits for the same token, and the launch
+// may pick either by batch size without changing any route.
+//
+// What changes is who does the work.  One warp owns a group of kGroupTokens
+// tokens and walks the eight virtual warps itself: per virtual warp its lanes
+// load the group's h chunks (the next virtual warp's loads are issued before
+// this one's arithmetic), read Wr's rows from shared memory (staged once per
+// CTA, shared by the group's tokens), and finish the virtual warp's sums with
+// a reduce-scatter over the same lane pairs as the xor tree (5 rounds, 31
+// shuffles for 32 (token, expert) sums), after which lane L holds token L / 8,
+// expert L % 8.  No warp waits for another after the prologue; four lanes run
+// the four tokens' top-k tails side by side.
+constexpr int kGroupTokens = 4;
+constexpr int kGroupThreads = 256;
+constexpr int kGroupMaxChunks = 4;                 // d <= 256 * 4 * 4 = 4096
+constexpr int64_t kGroupMinTokens = 64;           // smaller batches: pregate_kernel
+
+__host__ __device__ constexpr size_t group_smem_bytes(int64_t d) {
+    // Wr: one 4-row chunk (8 experts) per 9 float4 slots -- 8 of data, 1 of
+    // padding, so lanes reading their own chunks 144 bytes apart hit
+    // distinct bank groups
+    return (size_t)(d / 4) * 9 * 16;
+}
+
+template <int NCH>
+__global__ void __launch_bounds__(kGroupThreads, 1)
+pregate_group_kernel(const float* __restrict__ h, int64_t T, int64_t d,
+                     const float* __restrict__ Wr, int E, int k, int slots,
+                     int32_t* __restrict__ route, float* __restrict__ logits) {
+    extern __shared__ __align__(128) float4 wr_s[];
+    const int64_t nchunk = d >> 2;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr int TPB = kGroupTokens;
+
+    // ---- Wr into shared memory: chunk c's rows 4c..4c+3 (experts 0..7, zero
+    // past E) as float4 slots c * 9 + 2 * q + (e / 4), kStageBatch loads in
+    // flight per thread before their stores
+    {
+        constexpr int kStageBatch = 16;
+        const bool vec = E == 8 && (reinterpret_cast<uintptr_t>(Wr) & 15u) == 0;
+        const int64_t total = nchunk * 8;
+        for (int64_t i0 = threadIdx.x; i0 < total; i0 += kStageBatch * kGroupThreads) {
+            float4 v[kStageBatch];
+#pragma unroll
+            for (int u = 0; u < kStageBatch; ++u) {
+                const int64_t i = i0 + (int64_t)u * kGroupThreads;
+                const int64_t c = i >> 3;
+                const int f = (int)(i & 7);
+                if (i >= total) {
+                    v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                } else if (vec) {
+                    v[u] = __ldg(reinterpret_cast<const float4*>(Wr) + i);
+                } else {
+                    const int64_t row = 4 * c + (f >> 1);
+                    const int e0 = (f & 1) * 4;
+                    v[u].x = e0 + 0 < E ? __ldg(Wr + row * E + e0 + 0) : 0.f;
+                    v[u].y = e0 + 1 < E ? __ldg(Wr + row * E + e0 + 1) : 0.f;
+                    v[u].z = e0 + 2 < E ? __ldg(Wr + row * E + e0 + 2) : 0.f;
+                    v[u].w = e0 + 3 < E ? __ldg(Wr + row * E + e0 + 3) : 0.f;
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kStageBatch; ++u) {
+                const int64_t i = i0 + (int64_t)u * kGroupThreads;
+                if (i < total) wr_s[(i >> 3) * 9 + (i & 7)] = v[u];
+            }
+        }
+    }
+    __syncthreads();
+
+    const int64_t ngroups = (T + TPB - 1) / TPB;
+    const bool b16 = (lane & 16) != 0, b8 = (lane & 8) != 0, b4 = (lane & 4) != 0,
+               b2 = (lane & 2) != 0, b1 = (lane & 1) != 0;
+    // groups go round the CTAs first, so every SM gets a share of a batch
+    for (int64_t g = blockIdx.x + (int64_t)warp * gridDim.x; g < ngroups;
+         g += (int64_t)gridDim.x * (kGroupThreads / 32)) {
+        const int64_t t0 = g * TPB;
+        // h chunks of one virtual warp for the group's tokens (zero past T)
+        auto load_h = [&](int vw, float4 (&hv)[TPB][NCH]) {
+#pragma unroll
+            for (int m = 0; m < NCH; ++m) {
+                const int64_t c = 32 * vw + lane + 256 * m;
+#pragma unroll
+                for (int tt = 0; tt < TPB; ++tt)
+                    hv[tt][m] = (c < nchunk && t0 + tt < T)
+                                    ? __ldcs(reinterpret_cast<const float4*>(h + (t0 + tt) * d) + c)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        };
+        float4 ha[TPB][NCH], hb[TPB][NCH];
+        load_h(0, ha);
+        float zsum = 0.f;   // lane L: the in-order sum for token L / 8, expert L % 8
+#pragma unroll
+        for (int vw = 0; vw < 8; ++vw) {
+            float4 (&hc)[TPB][NCH] = (vw & 1) ? hb : ha;
+            float4 (&hn)[TPB][NCH] = (vw & 1) ? ha : hb;
+            if (vw + 1 < 8) load_h(vw + 1, hn);
+            float acc[TPB][8];
+#pragma unroll
+            for (int tt = 0; tt < TPB; ++tt)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[tt][e] = 0.f;
+#pragma unroll
+            for (int m = 0; m < NCH; ++m) {
+                const int64_t c = 32 * vw + lane + 256 * m;
+                if (c < nchunk) {
+                    float w[4][8];
+#pragma unroll
+                    for (int f = 0; f < 8; ++f) {
+                        const float4 v = wr_s[c * 9 + f];
+                        w[f >> 1][(f & 1) * 4 + 0] = v.x;
+                        w[f >> 1][(f & 1) * 4 + 1] = v.y;
+                        w[f >> 1][(f & 1) * 4 + 2] = v.z;
+                        w[f >> 1][(f & 1) * 4 + 3] = v.w;
+                    }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+#pragma unroll
+                            for (int tt = 0; tt < TPB; ++tt) {
+                                const float4 x4 = hc[tt][m];
+                                const float x = q == 0 ? x4.x : q == 1 ? x4.y : q == 2 ? x4.z : x4.w;
+                                acc[tt][e] = __fmaf_rn(x, w[q][e], acc[tt][e]);
+                            }
+                }
+            }
+            // the virtual warp's 32 sums (value index tt * 8 + e) by
+            // reduce-scatter: each round a lane keeps the half of its values
+            // its lane bit selects and adds its partner's copies of them, the
+            // pairs the xor tree adds; lane L ends with value L
+            float r16[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float lo = acc[i >> 3][i & 7], hi = acc[(16 + i) >> 3][(16 + i) & 7];
+                r16[i] = (b16 ? hi : lo) + __shfl_xor_sync(0xffffffffu, b16 ? lo : hi, 16);
+            }
+            float r8[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                r8[i] = (b8 ? r16[8 + i] : r16[i]) +
+                        __shfl_xor_sync(0xffffffffu, b8 ? r16[i] : r16[8 + i], 8);
+            float r4[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                r4[i] = (b4 ? r8[4 + i] : r8[i]) +
+                        __shfl_xor_sync(0xffffffffu, b4 ? r8[i] : r8[4 + i], 4);
+            float r2[2];
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+                r2[i] = (b2 ? r4[2 + i] : r4[i]) +
+                        __shfl_xor_sync(0xffffffffu, b2 ? r4[i] : r4[2 + i], 2);
+            const float r1 = (b1 ? r2[1] : r2[0]) + __shfl_xor_sync(0xffffffffu, b1 ? r2[0] : r2[1], 1);
+            zsum = vw == 0 ? r1 : zsum + r1;
+        }
+        // ---- the group's decisions: lane 8 * tt gathers token tt's logits
+        const int tt = lane >> 3, e = lane & 7;
+        const int64_t t = t0 + tt;
+        if (logits != nullptr) {
+            if (t < T && e < E) logits[t * E + e] = zsum;
+        } else {
+            float z[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) z[j] = __shfl_sync(0xffffffffu, zsum, (lane & ~7) + j);
+            if (e == 0 && t < T) route_tail<8>(z, E, k, slots, route, t);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// One routing decision for a decode batch: the kernels above, given a logits
+// buffer, write each token's fp32 logits z[t][0..E) there instead of its
+// route; this kernel (one CTA) then adds them in token order, divides by T
+// and applies the token rule (route_tail) to the mean.  With T = 1 the mean
+// is the token's own logits, bit for bit, so the batch route of one token is
+// its adafuse_pregate route.
+constexpr int kMaxBatchTokens = 4096;
+
+template <int EMAX>
+__global__ void __launch_bounds__(64)
+pregate_batch_reduce_kernel(const float* __restrict__ logits, int64_t T, int E, int k, int slots,
+                            int32_t* __restrict__ route) {
+    __shared__ float zbar[64];
+    const int e = threadIdx.x;
+    if (e < E) {
+        float v = logits[e];
+        for (int64_t t = 1; t < T; ++t) v += logits[t * E + e];
+        zbar[e] = v / (float)T;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float z[EMAX];
+#pragma unroll
+        for (int i = 0; i < EMAX; ++i) z[i] = i < E ? zbar[i] : 0.f;
+        route_tail<EMAX>(z, E, k, slots, route, 0);
     }
 }
 

@@ -266,7 +266,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_fold_kernel(const TcPara
                     uint8_t* a_dst = op_ring + (size_t)os * C::kOpStageBytes;
                     uint8_t* b_dst = a_dst + kFoldPairBytes;
                     mbar_arrive_expect_tx(&op_full[os], kFoldPairBytes + (has_b ? 2u : 1u) * bbytes +
-                                                            (p.stall && t == first && pr == 0 ? kStallBytes : 0u));
+                                                            (pr == 0 && (t - first) / gridDim.x + 1 == p.stall
+                                                                 ? kStallBytes : 0u));
                     bulk_load(a_dst, af + (size_t)pr * kFoldPairBytes, kFoldPairBytes, &op_full[os]);
                     const int ea = coef_expert(cf, 2 * pr);
                     bulk_load(b_dst, pd.Bk + ((size_t)ea * out + ti.row0) * 8, bbytes, &op_full[os]);

@@ -95,9 +95,11 @@ struct TcParams {
     // a tile is written even when no expert is selected (it copies W0).
     int rebase;
     const CUtensorMap* w0_maps;
-    // test hook: each CTA's first operand stage announces kStallBytes more
-    // than its loads deliver, so the MMA warp's bounded wait runs out and the
-    // launch ends through the timeout path before any MMA completes
+    // test hook (0 = off): the first operand stage of the stall-th tile each
+    // CTA (or CTA pair) processes announces kStallBytes more than its loads
+    // deliver, so the MMA warp's bounded wait runs out and the launch ends
+    // through the timeout path; the CTA's earlier tiles are finished and
+    // stored, that tile and later ones are not
     int stall;
     // tile schedule: 0 = static (CTA b takes tiles b, b + grid, ...); 1 =
     // dynamic (the W producers take tickets from sched[0] in table order, so
@@ -313,14 +315,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
             int os = 0, ts = 0;
             uint32_t oph = 0, tph = 0;
             uint32_t last_pair = 0xffffffffu;
-            bool first_tile = true;
+            int tile_no = 0;   // tiles this CTA has taken (for the stall hook)
             while (!*abort_flag) {
                 if (!mbar_wait_bounded(&te_full[ts], tph, abort_flag, kWaitLimitNs)) { fail(8); break; }
                 const TileEntry te = te_slot[ts];
                 if (++ts == C::kWStages) { ts = 0; tph ^= 1; }
                 if (te.x == kTileEndX) break;
-                const bool stall_here = p.stall && first_tile;
-                first_tile = false;
+                const bool stall_here = ++tile_no == p.stall;
                 const TileInfo ti = decode_tile(te);
                 const uint32_t pair = ti.pair;
                 const int row0 = ti.row0, col0 = ti.col0;

@@ -209,7 +209,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc2_kernel(const TcParam
                     uint8_t* b_dst = a_dst + C::kAHalfBytes;
                     const uint32_t full = full0 + 8u * (uint32_t)os;
                     mbar_arrive_expect_tx_cluster(
-                        full, bytes + (p.stall && q == 0 && t == first && ei == 0 ? kStallBytes : 0u));
+                        full, bytes + (q == 0 && ei == 0 && (t - first) / n_clusters + 1 == p.stall
+                                           ? kStallBytes : 0u));
                     if (ti.rows) tma_load_3d_pair(b_dst, mB, 0, ti.row0, e, full);
                     if (load_a) tma_load_3d_pair(a_dst, mA, ti.col0 + 64 * (int)q, 0, e, full);
                     if (++os == C::kOpStages) { os = 0; oph ^= 1; }
