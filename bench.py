@@ -82,6 +82,7 @@ KERNEL_SOURCES = {
                           "switch_tc_host.cuh"],
     "switch_fold_kernel": ["common.cuh", "sm100_ptx.cuh", "switch_tc.cuh", "switch_fold.cuh",
                            "switch_tc_host.cuh"],
+    "pregate_group_kernel": ["common.cuh", "sm100_ptx.cuh", "pregate.cuh"],
 }
 
 
@@ -902,6 +903,9 @@ def run_ours(args):
                   "hbm_gbs": round(r_bytes / (r_ms / 1e3) / 1e9, 1),
                   "frac_of_peak": round(r_bytes / (r_ms / 1e3) / 1e9 / measured_peaks()[0], 4),
                   "decode_token_ms_p50": round(dec_ms, 5),
+                  "kernel": "pregate_group_kernel" if (cfg.n_experts <= 8 and cfg.d <= 4096)
+                            else "pregate_kernel",
+                  "traffic": profiled_traffic("pregate_group_kernel", f"router-{Tr}x{cfg.d}-E{cfg.n_experts}"),
                   "l2": "flushed (256 MB write) before each timed batch launch"}
         del hr, rr
 

@@ -230,6 +230,26 @@ pregate_group_kernel(const float* __restrict__ h, int64_t T, int64_t d,
     const int64_t nchunk = d >> 2;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr int TPB = kGroupTokens;
+    const int64_t ngroups = (T + TPB - 1) / TPB;
+    // groups go round the CTAs first, so every SM gets a share of a batch
+    const int64_t g_first = blockIdx.x + (int64_t)warp * gridDim.x;
+    const int64_t g_step = (int64_t)gridDim.x * (kGroupThreads / 32);
+    // h chunks of one virtual warp for a group's tokens (zero past T)
+    auto load_h = [&](int64_t t0, int vw, float4 (&hv)[TPB][NCH]) {
+#pragma unroll
+        for (int m = 0; m < NCH; ++m) {
+            const int64_t c = 32 * vw + lane + 256 * m;
+#pragma unroll
+            for (int tt = 0; tt < TPB; ++tt)
+                hv[tt][m] = (c < nchunk && t0 + tt < T)
+                                ? __ldcs(reinterpret_cast<const float4*>(h + (t0 + tt) * d) + c)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    };
+    float4 ha[TPB][NCH], hb[TPB][NCH];
+    // the first group's first loads go out before Wr is staged, so the two
+    // latencies overlap
+    if (g_first < ngroups) load_h(g_first * TPB, 0, ha);
 
     // ---- Wr into shared memory: chunk c's rows 4c..4c+3 (experts 0..7, zero
     // past E) as float4 slots c * 9 + 2 * q + (e / 4), kStageBatch loads in
@@ -267,33 +287,17 @@ pregate_group_kernel(const float* __restrict__ h, int64_t T, int64_t d,
     }
     __syncthreads();
 
-    const int64_t ngroups = (T + TPB - 1) / TPB;
     const bool b16 = (lane & 16) != 0, b8 = (lane & 8) != 0, b4 = (lane & 4) != 0,
                b2 = (lane & 2) != 0, b1 = (lane & 1) != 0;
-    // groups go round the CTAs first, so every SM gets a share of a batch
-    for (int64_t g = blockIdx.x + (int64_t)warp * gridDim.x; g < ngroups;
-         g += (int64_t)gridDim.x * (kGroupThreads / 32)) {
+    for (int64_t g = g_first; g < ngroups; g += g_step) {
         const int64_t t0 = g * TPB;
-        // h chunks of one virtual warp for the group's tokens (zero past T)
-        auto load_h = [&](int vw, float4 (&hv)[TPB][NCH]) {
-#pragma unroll
-            for (int m = 0; m < NCH; ++m) {
-                const int64_t c = 32 * vw + lane + 256 * m;
-#pragma unroll
-                for (int tt = 0; tt < TPB; ++tt)
-                    hv[tt][m] = (c < nchunk && t0 + tt < T)
-                                    ? __ldcs(reinterpret_cast<const float4*>(h + (t0 + tt) * d) + c)
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-        };
-        float4 ha[TPB][NCH], hb[TPB][NCH];
-        load_h(0, ha);
+        if (g != g_first) load_h(t0, 0, ha);
         float zsum = 0.f;   // lane L: the in-order sum for token L / 8, expert L % 8
 #pragma unroll
         for (int vw = 0; vw < 8; ++vw) {
             float4 (&hc)[TPB][NCH] = (vw & 1) ? hb : ha;
             float4 (&hn)[TPB][NCH] = (vw & 1) ? ha : hb;
-            if (vw + 1 < 8) load_h(vw + 1, hn);
+            if (vw + 1 < 8) load_h(t0, vw + 1, hn);
             float acc[TPB][8];
 #pragma unroll
             for (int tt = 0; tt < TPB; ++tt)
