@@ -495,6 +495,7 @@ def config_leg(name, args, dev, stream, peak, peak_kind):
     then 3 warm-up and ``args.config_steps`` timed switches, with CUDA events
     around each launch on the launching stream.  Identity switches (prev ==
     cur bitwise) are timed apart and kept out of the roofline."""
+    import numpy as np
     import torch
     from weight_merge_b200 import binding as B
     from weight_merge_b200 import workloads as wl
@@ -516,7 +517,11 @@ def config_leg(name, args, dev, stream, peak, peak_kind):
         torch.cuda.synchronize()
         r_np = routes.cpu().numpy()
         warm, n = 3, max(10, args.config_steps)
-        seq = [k % T for k in range(warm + n)]
+        # where the sequence repeats a token (an identity switch, timed
+        # apart), the timed window is placed so that it holds the first one
+        rep = next((t for t in range(1, T) if np.array_equal(r_np[t], r_np[t - 1])), None)
+        start = 0 if rep is None else max(0, rep - warm - n // 2)
+        seq = [(start + k) % T for k in range(warm + n)]
         flags = moving_steps(r_np, seq, None)
         ptr = B.Switcher.route_ptr
         for k in range(warm):
