@@ -459,6 +459,8 @@ def e2e_leg(seq, prev_t, run_step, start, stop, read_routes, rebase=False):
     return ms, moving_steps(read_routes(), seq, prev_t, rebase), pe
 
 
+# adafuse_get_tensor_map_layout values (ADAFUSE_MAPS_NONE, _PLAIN, _BLOCKED)
+MAP_LAYOUTS = {0: "none", 1: "plain", 2: "blocked"}
 KERNEL_NAMES = {1: "switch_mma_kernel", 2: "switch_tc_kernel", 3: "switch_tc2_kernel",
                 4: "switch_fold_kernel"}
 
@@ -507,6 +509,7 @@ def config_leg(name, args, dev, stream, peak, peak_kind):
                     cfg.rank, cfg.alpha, device=dev, names=[t.name for t in cfg.targets])
     try:
         kind = sw.kernel
+        maps = MAP_LAYOUTS[sw.map_layout]
         T = cfg.n_tokens
         routes = route_buffer(cfg, T, False, "cuda")
         if routes is None:
@@ -555,6 +558,7 @@ def config_leg(name, args, dev, stream, peak, peak_kind):
         return {
             "workload": workload_label(cfg, T),
             "route_source": "router" if cfg.route_mode == "router" else f"synthesised ({cfg.route_mode})",
+            "tensor_maps": maps,
             "w_bytes_per_switch": w_bytes,
             "timed_switches": n,
             "switch_ms_p50": round(percentile(real, 0.5), 4),
@@ -734,6 +738,7 @@ def run_ours(args):
                     else B.ADAFUSE_SCHEDULE_STATIC)
     # the kernel this run's switches launch (in-place top-k calls have their own choice)
     kind = sw.topk_kernel if (args.top_k != 2 and args.mode != "rebase") else sw.kernel
+    maps = MAP_LAYOUTS[sw.map_layout]
     kernel_name = KERNEL_NAMES[kind]
     # the folded kernel's switch is two launches (fold, then switch); the
     # events around a switch cover both
@@ -971,6 +976,7 @@ def run_ours(args):
                 "mode": args.mode,
                 "route_source": "router" if synth is None else f"synthesised ({cfg.route_mode})",
                 "tile_schedule": args.schedule if kind == B.ADAFUSE_KERNEL_TCGEN05 else "static",
+                "tensor_maps": maps,
             },
             "switch_ms_p50": round(sw_sorted[len(sw_sorted) // 2], 4),
             "switch_ms_p90": round(sw_sorted[min(len(sw_sorted) - 1, int(0.9 * len(sw_sorted)))], 4),

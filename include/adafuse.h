@@ -105,6 +105,14 @@ extern "C" {
 #define ADAFUSE_SCHEDULE_STATIC  0
 #define ADAFUSE_SCHEDULE_DYNAMIC 1
 
+/* ---- TMA tensor-map layouts (adafuse_get_tensor_map_layout) ------------- */
+#define ADAFUSE_MAPS_NONE    0  /* no tensor maps: only the mma.sync kernel runs */
+#define ADAFUSE_MAPS_PLAIN   1  /* some weight's in is not a multiple of 64: a 128 x 128
+                                   W tile moves as two 64-column TMA operations */
+#define ADAFUSE_MAPS_BLOCKED 2  /* every in a multiple of 64: W viewed as 64-column
+                                   blocks, one TMA operation per W tile load or store
+                                   and per expert's A columns */
+
 /* One token's routing decision: the two chosen experts and their gates.
  * idx[j] == -1 marks an empty slot (its gate is ignored).  adafuse_pregate
  * writes gate[0] >= gate[1], gate[0] + gate[1] == 1 (up to rounding). */
@@ -253,6 +261,12 @@ ADAFUSE_API int adafuse_set_max_ctas(adafuse_ctx* ctx, int32_t max_ctas);
  * ADAFUSE_KERNEL_TCGEN05, ADAFUSE_KERNEL_TCGEN05_PAIR or
  * ADAFUSE_KERNEL_TCGEN05_FOLD), or a negative code. */
 ADAFUSE_API int adafuse_get_switch_kernel(adafuse_ctx* ctx);
+
+/* The tensor-map layout adafuse_create chose for this context
+ * (ADAFUSE_MAPS_NONE, _PLAIN or _BLOCKED), or a negative code.  The layout
+ * changes how many TMA operations move a tile, never a result: the same
+ * elements are read and written either way, so W is bit for bit the same. */
+ADAFUSE_API int adafuse_get_tensor_map_layout(const adafuse_ctx* ctx);
 
 /* ---- re-base switch ------------------------------------------------------
  * A variant of the switch that the AdaFuse pages do not describe (they merge

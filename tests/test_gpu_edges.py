@@ -203,20 +203,28 @@ def test_bounded_wait_timeout_reports_status_and_context_stays_usable(kernel, r)
     _switch_and_check(cfg, m, sw, routes, [(None, 0), (0, 1)])
 
 
+MID_SHAPES = {"blocked": [("q", 1024, 1024), ("o", 1280, 768)],
+              "plain": [("q", 1024, 1032), ("o", 1280, 776)]}
+
+
+@pytest.mark.parametrize("layout", ["blocked", "plain"])
 @pytest.mark.parametrize("kernel,r", [(TC, 8), (TC2, 16), (TF, 8), (TC, 32)])
-def test_timeout_mid_launch_leaves_whole_tiles_and_rebase_recovers(kernel, r):
+def test_timeout_mid_launch_leaves_whole_tiles_and_rebase_recovers(kernel, r, layout):
     """A bounded wait that runs out in the middle of a switch: the hook
     stalls each CTA's second tile, so every CTA stores its first tile and
     stops.  Every 128 x 128 tile must then be either untouched or fully
     switched (the oracle's prev -> cur result), with both kinds present; the
     documented recovery, a re-base from the registered pristine weights,
     gives the oracle's W0 + dW(cur) everywhere."""
-    cfg = wl.custom("mid", 2, [("q", 1024, 1024), ("o", 1280, 768)], n_experts=4, rank=r,
-                    alpha=2.0 * r, n_tokens=2, d=1024)
+    shapes = MID_SHAPES[layout]
+    cfg = wl.custom("mid", 2, shapes, n_experts=4, rank=r, alpha=2.0 * r, n_tokens=2,
+                    d=shapes[0][2])
     m = wl.make_model(cfg, device="cuda", seed=90 + r)
     sw = Bnd.Switcher(m.W, m.A, m.B, cfg.n_layers, len(cfg.targets), cfg.n_experts, cfg.rank,
                       cfg.alpha, device=torch.cuda.current_device())
     sw.set_kernel(kernel)
+    assert sw.map_layout == (Bnd.ADAFUSE_MAPS_BLOCKED if layout == "blocked"
+                             else Bnd.ADAFUSE_MAPS_PLAIN)
     base = [w.clone() for w in m.W]
     sw.set_base(base)
     W0 = [bits(w) for w in base]

@@ -193,17 +193,26 @@ def test_tiny_sequence_lockstep_all_elements():
 
 
 RAGGED = [("a", 200, 136), ("b", 8, 8), ("c", 264, 392), ("d", 128, 256), ("e", 136, 8)]
+# every in a multiple of 64, so the context takes blocked tensor maps; in = 192,
+# 64 and 320 end on a half-width (64-column) tile
+RAGGED_BLOCKED = [("a", 200, 192), ("b", 8, 64), ("c", 264, 320), ("d", 128, 256), ("e", 136, 64)]
+SHAPE_SETS = {"plain": (RAGGED, Bnd.ADAFUSE_MAPS_PLAIN),
+              "blocked": (RAGGED_BLOCKED, Bnd.ADAFUSE_MAPS_BLOCKED)}
 
 
 RANKS = [(1, 1), (3, 3), (4, 4), (5, 8), (16, 12), (4, 16), (6, 24), (3, 32), (4, 40), (5, 64)]
 
 
+@pytest.mark.parametrize("layout", sorted(SHAPE_SETS))
 @pytest.mark.parametrize("E,r,kernel", [(E, r, k) for (E, r) in RANKS for k in kernels_for(r)])
-def test_ragged_shapes_every_rank_class(E, r, kernel):
-    cfg = wl.custom("ragged", 2, RAGGED, n_experts=E, rank=r, alpha=2.0 * r, n_tokens=6,
-                    d=136)
+def test_ragged_shapes_every_rank_class(E, r, kernel, layout):
+    shapes, want_layout = SHAPE_SETS[layout]
+    cfg = wl.custom("ragged", 2, shapes, n_experts=E, rank=r, alpha=2.0 * r, n_tokens=6,
+                    d=shapes[0][2])
     model = wl.make_model(cfg, device="cuda", seed=1000 + 7 * r + E)
     sw = make_switcher(model, kernel)
+    if kernel != MMA:
+        assert sw.map_layout == want_layout
     rng = np.random.default_rng(r * 31 + E)
     T = 6
     idx = rng.integers(0, E, size=(T, 2)).astype(np.int32)

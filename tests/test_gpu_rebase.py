@@ -21,6 +21,8 @@ pytestmark = pytest.mark.gpu
 MMA, TC, TC2, TF = (Bnd.ADAFUSE_KERNEL_MMA_SYNC, Bnd.ADAFUSE_KERNEL_TCGEN05,
                     Bnd.ADAFUSE_KERNEL_TCGEN05_PAIR, Bnd.ADAFUSE_KERNEL_TCGEN05_FOLD)
 SHAPES = [("a", 200, 136), ("b", 264, 392), ("c", 128, 256), ("d", 8, 8)]
+# every in a multiple of 64 (blocked tensor maps), half-width last tiles
+SHAPES_BLOCKED = [("a", 200, 192), ("b", 264, 320), ("c", 128, 256), ("d", 8, 64)]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -56,12 +58,16 @@ def _check_against_oracle(cfg, m, W0, route, A_h, B_h):
                           None, route)
 
 
+@pytest.mark.parametrize("blocked", [False, True])
 @pytest.mark.parametrize("E,r,kernel", [(3, 3, MMA), (4, 8, MMA), (4, 8, TC), (5, 16, TC),
                                         (3, 24, MMA), (4, 32, TC), (6, 64, TC), (5, 16, TC2),
                                         (3, 24, TC2), (4, 32, TC2), (6, 64, TC2), (3, 3, TC),
                                         (4, 4, TC), (4, 8, TF), (3, 3, TF)])
-def test_rebase_matches_oracle_and_does_not_accumulate(E, r, kernel):
-    cfg, m, sw, W0 = _setup(E, r, kernel, seed=31 * r + E)
+def test_rebase_matches_oracle_and_does_not_accumulate(E, r, kernel, blocked):
+    cfg, m, sw, W0 = _setup(E, r, kernel, seed=31 * r + E,
+                            shapes=SHAPES_BLOCKED if blocked else SHAPES)
+    if kernel != MMA:
+        assert sw.map_layout == (Bnd.ADAFUSE_MAPS_BLOCKED if blocked else Bnd.ADAFUSE_MAPS_PLAIN)
     W0_bits = [bits(w) for w in W0]
     A_h = [bits(a) for a in m.A]
     B_h = [bits(b) for b in m.B]

@@ -132,6 +132,8 @@ def test_pregate_topk_rejects_bad_k():
 # the switch with top-k routes
 
 RAGGED = [("a", 200, 136), ("b", 8, 8), ("c", 264, 392), ("d", 128, 256), ("e", 136, 8)]
+# blocked tensor maps (every in a multiple of 64), half-width last tiles
+RAGGED_BLOCKED = [("a", 200, 192), ("b", 8, 64), ("c", 264, 320), ("d", 128, 256), ("e", 136, 64)]
 RANKS = [(9, 4), (9, 8), (9, 16), (9, 24), (10, 64)]
 
 
@@ -183,12 +185,16 @@ def _ragged_routes(E, seed):
     return idx, gate
 
 
+@pytest.mark.parametrize("blocked", [False, True])
 @pytest.mark.parametrize("E,r,kernel", [(E, r, k) for (E, r) in RANKS for k in kernels_for(r)])
-def test_switch_topk_ragged_shapes_every_kernel(E, r, kernel):
-    cfg = wl.custom("ragged", 2, RAGGED, n_experts=E, rank=r, alpha=2.0 * r, n_tokens=7, d=136)
+def test_switch_topk_ragged_shapes_every_kernel(E, r, kernel, blocked):
+    shapes = RAGGED_BLOCKED if blocked else RAGGED
+    cfg = wl.custom("ragged", 2, shapes, n_experts=E, rank=r, alpha=2.0 * r, n_tokens=7,
+                    d=shapes[0][2])
     model = wl.make_model(cfg, device="cuda", seed=3000 + 7 * r + E)
     sw = switcher(model, kernel)
     assert sw.kernel == kernel
+    assert sw.map_layout == (Bnd.ADAFUSE_MAPS_BLOCKED if blocked else Bnd.ADAFUSE_MAPS_PLAIN)
     idx, gate = _ragged_routes(E, seed=r * 13 + E)
     routes = make_routes4(idx, gate)
     A_h, B_h = [bits(a) for a in model.A], [bits(b) for b in model.B]

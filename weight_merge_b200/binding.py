@@ -31,6 +31,9 @@ ADAFUSE_KERNEL_TCGEN05_PAIR = 3
 ADAFUSE_KERNEL_TCGEN05_FOLD = 4
 ADAFUSE_SCHEDULE_STATIC = 0
 ADAFUSE_SCHEDULE_DYNAMIC = 1
+ADAFUSE_MAPS_NONE = 0
+ADAFUSE_MAPS_PLAIN = 1
+ADAFUSE_MAPS_BLOCKED = 2
 ADAFUSE_MAX_TOP_K = 4
 ADAFUSE_MAX_BATCH_TOKENS = 4096
 
@@ -97,6 +100,7 @@ def lib() -> ctypes.CDLL:
         "adafuse_rebase": ([P, P, P], ctypes.c_int),
         "adafuse_rebase_layers": ([P, i32, i32, P, P], ctypes.c_int),
         "adafuse_get_switch_kernel": ([P], ctypes.c_int),
+        "adafuse_get_tensor_map_layout": ([P], ctypes.c_int),
         "adafuse_pregate_topk": ([P, P, i64, i64, P, i32, P, P], ctypes.c_int),
         "adafuse_pregate_batch": ([P, P, i64, i64, P, P, P], ctypes.c_int),
         "adafuse_pregate_batch_topk": ([P, P, i64, i64, P, i32, P, P], ctypes.c_int),
@@ -253,6 +257,13 @@ def adafuse_get_switch_kernel(ctx: int) -> int:
     return k
 
 
+def adafuse_get_tensor_map_layout(ctx: int) -> int:
+    k = lib().adafuse_get_tensor_map_layout(ctx)
+    if k < 0:
+        raise AdafuseError(k, "adafuse_get_tensor_map_layout")
+    return k
+
+
 def adafuse_get_device_status(ctx: int, stream: int = 0, raise_on_fault: bool = False) -> int:
     v = ctypes.c_int32(0)
     code = lib().adafuse_get_device_status(ctx, stream or None, ctypes.byref(v))
@@ -387,6 +398,10 @@ class Switcher:
     @property
     def kernel(self) -> int:
         return adafuse_get_switch_kernel(self.ctx)
+
+    @property
+    def map_layout(self) -> int:
+        return adafuse_get_tensor_map_layout(self.ctx)
 
     @property
     def topk_kernel(self) -> int:

@@ -31,7 +31,8 @@ struct adafuse_ctx {
     PairDesc* d_pairs = nullptr;
     TileEntry* d_tiles = nullptr;
     int32_t* d_status = nullptr;
-    CUtensorMap* d_maps = nullptr;  // 3 per pair (W, A, B) when the tensor-core kernel can run
+    CUtensorMap* d_maps = nullptr;  // kMapsPerPair per pair when the tensor-core kernel can run
+    bool blk = false;               // those maps are blocked (every weight's in % 64 == 0)
     int tc_kp = 0;                  // its padded rank (16, 32, 64), 0 = not eligible
     int kernel = ADAFUSE_KERNEL_AUTO;
     std::vector<PairDesc> h_pairs;  // host copy of d_pairs (re-base pointers are patched in)
@@ -251,6 +252,7 @@ cudaError_t launch_tc(adafuse_ctx* c, int64_t t0, int64_t t1, const int32_t* pre
     prm.pairs = c->d_pairs;
     prm.tiles = c->d_tiles;
     prm.maps = c->d_maps;
+    prm.blk = c->blk ? 1 : 0;
     prm.t_begin = t0;
     prm.t_end = t1;
     prm.prev = prev;
@@ -282,6 +284,7 @@ cudaError_t launch_tc2(adafuse_ctx* c, int64_t b0, int64_t b1, const int32_t* pr
     prm.pairs = c->d_pairs;
     prm.tiles = c->d_blocks;
     prm.maps = c->d_maps;
+    prm.blk = c->blk ? 1 : 0;
     prm.t_begin = b0;
     prm.t_end = b1;
     prm.prev = prev;
@@ -467,13 +470,25 @@ int adafuse_create(adafuse_ctx** out, const adafuse_desc* desc, int device) {
         bool ok = enc != nullptr;
         if (ok) {
             try {
-                maps.resize((size_t)npairs * 3);
+                maps.resize((size_t)npairs * kMapsPerPair);
             } catch (...) {
                 ok = false;
             }
         }
-        for (int64_t i = 0; ok && i < npairs; ++i)
-            ok = encode_pair_maps(enc, pairs[i], desc->n_experts, desc->rank, c->tc_kp, &maps[3 * i]);
+        // blocked maps where every weight allows them; plain ones if the
+        // driver refuses a blocked encoding
+        c->blk = blocked_maps_ok(pairs.data(), npairs);
+        for (int pass = 0; pass < 2; ++pass) {
+            bool enc_ok = ok;
+            for (int64_t i = 0; enc_ok && i < npairs; ++i)
+                enc_ok = encode_pair_maps(enc, pairs[i], desc->n_experts, desc->rank, c->tc_kp,
+                                          c->blk, &maps[kMapsPerPair * i]);
+            if (enc_ok || !c->blk) {
+                ok = ok && enc_ok;
+                break;
+            }
+            c->blk = false;
+        }
         if (ok) {
             if ((e = cudaMalloc(&c->d_maps, sizeof(CUtensorMap) * maps.size())) != cudaSuccess)
                 return fail(e, "cudaMalloc(maps)");
@@ -570,6 +585,11 @@ int adafuse_set_max_ctas(adafuse_ctx* ctx, int32_t max_ctas) {
     if (ctx == nullptr || max_ctas < 0) return ADAFUSE_ERR_INVALID_ARG;
     ctx->max_ctas = max_ctas;
     return ADAFUSE_OK;
+}
+
+int adafuse_get_tensor_map_layout(const adafuse_ctx* ctx) {
+    if (ctx == nullptr) return ADAFUSE_ERR_INVALID_ARG;
+    return ctx->tc_kp == 0 ? ADAFUSE_MAPS_NONE : ctx->blk ? ADAFUSE_MAPS_BLOCKED : ADAFUSE_MAPS_PLAIN;
 }
 
 int adafuse_get_switch_kernel(adafuse_ctx* ctx) {
@@ -774,6 +794,7 @@ int launch_switch(adafuse_ctx* ctx, int32_t layer_begin, int32_t n_layers,
         prm.pairs = ctx->d_pairs;
         prm.tiles = ctx->d_tiles;
         prm.maps = ctx->d_maps;
+        prm.blk = ctx->blk ? 1 : 0;
         prm.t_begin = t0;
         prm.t_end = t1;
         prm.prev = prev;
@@ -857,12 +878,8 @@ int adafuse_set_base(adafuse_ctx* ctx, const void* const* W0) {
         EncodeTiledFn enc = encode_tiled_fn();
         if (enc == nullptr) return ADAFUSE_ERR_CUDA;
         for (size_t i = 0; i < n; ++i) {
-            PairDesc src = pairs[i];
-            src.W = const_cast<uint16_t*>(src.W0);
-            CUtensorMap three[3];
-            if (!encode_pair_maps(enc, src, ctx->n_experts, ctx->rank, ctx->tc_kp, three))
+            if (!encode_w_map(enc, pairs[i].W0, pairs[i].out, pairs[i].in, ctx->blk, &maps[i]))
                 return ADAFUSE_ERR_CUDA;
-            maps[i] = three[0];
         }
     }
     // everything the kernels may still be reading is replaced only after the

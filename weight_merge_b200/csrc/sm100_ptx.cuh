@@ -104,6 +104,23 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const void* map, int32_t 
         : "memory");
 }
 
+__device__ __forceinline__ void tma_load_4d(void* dst, const void* map, int32_t x, int32_t y,
+                                            int32_t z, int32_t w, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_store_3d(const void* map, const void* src, int32_t x,
+                                             int32_t y, int32_t z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(map),
+        "r"(x), "r"(y), "r"(z), "r"(smem_u32(src))
+        : "memory");
+}
+
 __device__ __forceinline__ void tma_store_2d(const void* map, const void* src, int32_t x,
                                              int32_t y) {
     asm volatile(

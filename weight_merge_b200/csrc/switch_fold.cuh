@@ -223,20 +223,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_fold_kernel(const TcPara
             for (int64_t t = first; t < p.t_end && !*abort_flag; t += gridDim.x) {
                 const TileInfo ti = decode_tile(te_next);
                 te_next = fetch_tile(p.tiles, t + gridDim.x, p.t_end);
-                const CUtensorMap* mW = p.rebase ? p.w0_maps + ti.pair : p.maps + 3 * (size_t)ti.pair;
+                const CUtensorMap* mW = p.rebase ? p.w0_maps + ti.pair : p.maps + kMapsPerPair * (size_t)ti.pair;
                 if (ti.pair != last_pair) {
                     tensormap_acquire(mW);
                     last_pair = ti.pair;
                 }
                 if (!mbar_wait_bounded(&w_empty[ws], wph ^ 1, abort_flag, kWaitLimitNs)) { fail(1); break; }
                 uint8_t* wdst = w_ring + (size_t)ws * kWTileBytes;
-                mbar_arrive_expect_tx(&w_full[ws], ti.wide ? kWTileBytes : kWBoxBytes);
-                tma_load_2d(wdst, mW, ti.col0, ti.row0, &w_full[ws]);
-                if (ti.wide) tma_load_2d(wdst + kWBoxBytes, mW, ti.col0 + 64, ti.row0, &w_full[ws]);
+                mbar_arrive_expect_tx(&w_full[ws], w_tile_bytes(p.blk, ti.wide));
+                load_w_tile(wdst, mW, ti.row0, ti.col0, ti.wide, p.blk, &w_full[ws]);
                 if (++ws == C::kWStages) { ws = 0; wph ^= 1; }
                 if (t + gridDim.x < p.t_end && (te_next.x & kTilePairMask) != ti.pair) {
                     const uint32_t np = te_next.x & kTilePairMask;
-                    tensormap_prefetch(p.rebase ? p.w0_maps + np : p.maps + 3 * (size_t)np);
+                    tensormap_prefetch(p.rebase ? p.w0_maps + np : p.maps + kMapsPerPair * (size_t)np);
                 }
             }
         }
@@ -332,10 +331,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_fold_kernel(const TcPara
                 const TileInfo ti = decode_tile(te_next);
                 te_next = fetch_tile(p.tiles, t + gridDim.x, p.t_end);
                 if (!mbar_wait_bounded(&epi_done[ws], wph, abort_flag, kWaitLimitNs)) { fail(7); break; }
-                const CUtensorMap* mW = p.maps + 3 * (size_t)ti.pair;
+                const CUtensorMap* mW = p.maps + kMapsPerPair * (size_t)ti.pair;
                 uint8_t* wsrc = w_ring + (size_t)ws * kWTileBytes;
-                tma_store_2d(mW, wsrc, ti.col0, ti.row0);
-                if (ti.wide) tma_store_2d(mW, wsrc + kWBoxBytes, ti.col0 + 64, ti.row0);
+                store_w_tile(mW, wsrc, ti.row0, ti.col0, ti.wide, p.blk);
                 bulk_commit();
                 bulk_wait_read<0>();
                 mbar_arrive(&w_empty[ws]);

@@ -79,10 +79,48 @@ struct TcConfig {
     static_assert(kOpStageBytes % 1024 == 0 && kAHalfBytes % 1024 == 0, "swizzle atoms stay aligned");
 };
 
+// Tensor maps per (layer, target): W, A, B, and A as 64-column blocks.
+//   plain (some weight's in is not a multiple of 64): W [out, in] with a
+//     64 x 128 box (two loads or stores per 128 x 128 tile), A [E, r, in]
+//     with a 64 x rows box (two loads per expert and tile);
+//   blocked (every in a multiple of 64): W as [in/64 blocks][out][64] with a
+//     64 x 128 x 2 box and A as [E][in/64][r][64] with a 64 x rows x 2 x 1
+//     box, so one TMA operation moves a whole tile's W or an expert's A
+//     columns into the same shared-memory layout (blocks 16 KB / 1 KB apart).
+//     The number of TMA operations per tile is a measured cost of these
+//     kernels.  Slot 1 keeps the plain A map, which the pair kernel uses.
+constexpr int kMapsPerPair = 4;
+
+// One W tile (128 rows x 128 columns at (row0, col0)): the bytes its load
+// brings, the load and the store.  A half past the weight's last column is
+// zero-filled on load (blocked) or not loaded (plain), and never stored.
+__device__ __forceinline__ uint32_t w_tile_bytes(bool blk, bool wide) {
+    return (blk || wide) ? kWTileBytes : kWBoxBytes;
+}
+__device__ __forceinline__ void load_w_tile(void* dst, const CUtensorMap* m, int row0, int col0,
+                                            bool wide, bool blk, uint64_t* bar) {
+    if (blk) {
+        sm100::tma_load_3d(dst, m, 0, row0, col0 >> 6, bar);
+    } else {
+        sm100::tma_load_2d(dst, m, col0, row0, bar);
+        if (wide) sm100::tma_load_2d(static_cast<uint8_t*>(dst) + kWBoxBytes, m, col0 + 64, row0, bar);
+    }
+}
+__device__ __forceinline__ void store_w_tile(const CUtensorMap* m, const void* src, int row0,
+                                             int col0, bool wide, bool blk) {
+    if (blk) {
+        sm100::tma_store_3d(m, src, 0, row0, col0 >> 6);
+    } else {
+        sm100::tma_store_2d(m, src, col0, row0);
+        if (wide) sm100::tma_store_2d(m, static_cast<const uint8_t*>(src) + kWBoxBytes, col0 + 64, row0);
+    }
+}
+
 struct TcParams {
     const PairDesc* pairs;
     const TileEntry* tiles;
-    const CUtensorMap* maps;  // 3 per pair: W, A, B
+    const CUtensorMap* maps;  // kMapsPerPair per pair: W, A, B, A as 64-column blocks
+    int blk;                  // 1: blocked maps (see kMapsPerPair)
     int64_t t_begin, t_end;
     const int32_t* prev;  // routes of `slots` slots (adafuse_route or adafuse_route4)
     const int32_t* cur;
@@ -288,21 +326,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
                 te_slot[ws] = te;
                 mbar_arrive(&te_full[ws]);
                 const TileInfo ti = decode_tile(te);
-                const CUtensorMap* mW = p.rebase ? p.w0_maps + ti.pair : p.maps + 3 * (size_t)ti.pair;
+                const CUtensorMap* mW = p.rebase ? p.w0_maps + ti.pair : p.maps + kMapsPerPair * (size_t)ti.pair;
                 if (ti.pair != last_pair) {
                     tensormap_acquire(mW);
                     last_pair = ti.pair;
                 }
                 uint8_t* wdst = w_ring + (size_t)ws * kWTileBytes;
-                mbar_arrive_expect_tx(&w_full[ws], ti.wide ? kWTileBytes : kWBoxBytes);
-                tma_load_2d(wdst, mW, ti.col0, ti.row0, &w_full[ws]);
-                if (ti.wide) tma_load_2d(wdst + kWBoxBytes, mW, ti.col0 + 64, ti.row0, &w_full[ws]);
+                mbar_arrive_expect_tx(&w_full[ws], w_tile_bytes(p.blk, ti.wide));
+                load_w_tile(wdst, mW, ti.row0, ti.col0, ti.wide, p.blk, &w_full[ws]);
                 if (++ws == C::kWStages) { ws = 0; wph ^= 1; }
                 if (tn < p.t_end && (te_n.x & kTilePairMask) != ti.pair) {
                     const uint32_t np = te_n.x & kTilePairMask;
-                    tensormap_prefetch(p.rebase ? p.w0_maps + np : p.maps + 3 * (size_t)np);
-                    tensormap_prefetch(p.maps + 3 * (size_t)np + 1);
-                    tensormap_prefetch(p.maps + 3 * (size_t)np + 2);
+                    const CUtensorMap* nm = p.maps + kMapsPerPair * (size_t)np;
+                    tensormap_prefetch(p.rebase ? p.w0_maps + np : nm);
+                    tensormap_prefetch(nm + (p.blk ? 3 : 1));
+                    tensormap_prefetch(nm + 2);
                 }
                 t = tn;
                 te = te_n;
@@ -325,14 +363,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
                 const TileInfo ti = decode_tile(te);
                 const uint32_t pair = ti.pair;
                 const int row0 = ti.row0, col0 = ti.col0;
-                const CUtensorMap* mA = p.maps + 3 * (size_t)pair + 1;
-                const CUtensorMap* mB = mA + 1;
+                const CUtensorMap* mA = p.maps + kMapsPerPair * (size_t)pair + (p.blk ? 3 : 1);
+                const CUtensorMap* mB = p.maps + kMapsPerPair * (size_t)pair + 2;
                 if (pair != last_pair) {
                     tensormap_acquire(mA);
                     tensormap_acquire(mB);
                     last_pair = pair;
                 }
                 const bool second = ti.wide;
+                // A columns of one expert: one blocked load of both 64-column
+                // halves, or one plain load per half inside the weight
+                const uint32_t a_bytes = (p.blk || second) ? 2 * C::kAHalfBytes : C::kAHalfBytes;
                 int out_rows = 128;
                 const uint16_t* Bbase = nullptr;
                 int out = 0;
@@ -353,16 +394,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
                         // rows past the weight's end are not fetched (their
                         // products only reach accumulator rows never stored)
                         const uint32_t bbytes = (uint32_t)out_rows * 16u;
-                        mbar_arrive_expect_tx(&op_full[os], bbytes + (second ? 2 : 1) * C::kAHalfBytes +
+                        mbar_arrive_expect_tx(&op_full[os], bbytes + a_bytes +
                                                                 (stall_here && ei == 0 ? kStallBytes : 0u));
                         bulk_load(b_dst, Bbase + ((size_t)e * out + row0) * 8, bbytes, &op_full[os]);
                     } else {
-                        mbar_arrive_expect_tx(&op_full[os], C::kBBytes + (second ? 2 : 1) * C::kAHalfBytes +
+                        mbar_arrive_expect_tx(&op_full[os], C::kBBytes + a_bytes +
                                                                 (stall_here && ei == 0 ? kStallBytes : 0u));
                         tma_load_3d(b_dst, mB, 0, row0, e, &op_full[os]);
                     }
-                    tma_load_3d(a_dst, mA, col0, 0, e, &op_full[os]);
-                    if (second) tma_load_3d(a_dst + C::kAHalfBytes, mA, col0 + 64, 0, e, &op_full[os]);
+                    if (p.blk) {
+                        tma_load_4d(a_dst, mA, 0, 0, col0 >> 6, e, &op_full[os]);
+                    } else {
+                        tma_load_3d(a_dst, mA, col0, 0, e, &op_full[os]);
+                        if (second) tma_load_3d(a_dst + C::kAHalfBytes, mA, col0 + 64, 0, e, &op_full[os]);
+                    }
                     if (++os == C::kOpStages) { os = 0; oph ^= 1; }
                 }
                 if (!ok) { fail(2); break; }
@@ -439,11 +484,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc_kernel(const TcParams
                     const TileInfo ti = decode_tile(te);
                     const int row0 = ti.row0, col0 = ti.col0;
                     if (!mbar_wait_bounded(&epi_done[ws], wph, abort_flag, kWaitLimitNs)) { fail(7); break; }
-                    const CUtensorMap* mW = p.maps + 3 * (size_t)ti.pair;
-                    const bool second = ti.wide;
+                    const CUtensorMap* mW = p.maps + kMapsPerPair * (size_t)ti.pair;
                     uint8_t* wsrc = w_ring + (size_t)ws * kWTileBytes;
-                    tma_store_2d(mW, wsrc, col0, row0);
-                    if (second) tma_store_2d(mW, wsrc + kWBoxBytes, col0 + 64, row0);
+                    store_w_tile(mW, wsrc, row0, col0, ti.wide, p.blk);
                     bulk_commit();
                     bulk_wait_read<0>();
                     mbar_arrive(&w_empty[ws]);

@@ -156,7 +156,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc2_kernel(const TcParam
             for (int64_t t = first; t < p.t_end && !*abort_flag; t += n_clusters) {
                 const PairTile ti = decode_pair_tile(te_next, q);
                 te_next = fetch_tile(p.tiles, t + n_clusters, p.t_end);
-                const CUtensorMap* mW = p.rebase ? p.w0_maps + ti.pair : p.maps + 3 * (size_t)ti.pair;
+                const CUtensorMap* mW = p.rebase ? p.w0_maps + ti.pair : p.maps + kMapsPerPair * (size_t)ti.pair;
                 if (ti.pair != last_pair) {
                     tensormap_acquire(mW);
                     last_pair = ti.pair;
@@ -164,9 +164,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc2_kernel(const TcParam
                 if (!mbar_wait_bounded(&w_empty[ws], wph ^ 1, abort_flag, kWaitLimitNs)) { fail(1); break; }
                 uint8_t* wdst = w_ring + (size_t)ws * kWTileBytes;
                 if (ti.rows) {
-                    mbar_arrive_expect_tx(&w_full[ws], ti.wide ? kWTileBytes : kWBoxBytes);
-                    tma_load_2d(wdst, mW, ti.col0, ti.row0, &w_full[ws]);
-                    if (ti.wide) tma_load_2d(wdst + kWBoxBytes, mW, ti.col0 + 64, ti.row0, &w_full[ws]);
+                    mbar_arrive_expect_tx(&w_full[ws], w_tile_bytes(p.blk, ti.wide));
+                    load_w_tile(wdst, mW, ti.row0, ti.col0, ti.wide, p.blk, &w_full[ws]);
                 } else {
                     // no rows of this weight here: the stage is only passed along
                     mbar_arrive(&w_full[ws]);
@@ -174,7 +173,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc2_kernel(const TcParam
                 if (++ws == C::kWStages) { ws = 0; wph ^= 1; }
                 if (t + n_clusters < p.t_end && (te_next.x & kTile2PairMask) != ti.pair) {
                     const uint32_t np = te_next.x & kTile2PairMask;
-                    tensormap_prefetch(p.rebase ? p.w0_maps + np : p.maps + 3 * (size_t)np);
+                    tensormap_prefetch(p.rebase ? p.w0_maps + np : p.maps + kMapsPerPair * (size_t)np);
                 }
             }
         }
@@ -192,7 +191,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc2_kernel(const TcParam
             for (int64_t t = first; t < p.t_end && !*abort_flag; t += n_clusters) {
                 const PairTile ti = decode_pair_tile(te_next, q);
                 te_next = fetch_tile(p.tiles, t + n_clusters, p.t_end);
-                const CUtensorMap* mA = p.maps + 3 * (size_t)ti.pair + 1;
+                const CUtensorMap* mA = p.maps + kMapsPerPair * (size_t)ti.pair + 1;
                 const CUtensorMap* mB = mA + 1;
                 if (ti.pair != last_pair) {
                     tensormap_acquire(mA);
@@ -217,7 +216,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc2_kernel(const TcParam
                 }
                 if (!ok) { fail(2); break; }
                 if (t + n_clusters < p.t_end && (te_next.x & kTile2PairMask) != ti.pair) {
-                    const CUtensorMap* nm = p.maps + 3 * (size_t)(te_next.x & kTile2PairMask);
+                    const CUtensorMap* nm = p.maps + kMapsPerPair * (size_t)(te_next.x & kTile2PairMask);
                     tensormap_prefetch(nm + 1);
                     tensormap_prefetch(nm + 2);
                 }
@@ -279,10 +278,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc2_kernel(const TcParam
                 te_next = fetch_tile(p.tiles, t + n_clusters, p.t_end);
                 if (!mbar_wait_bounded(&epi_done[ws], wph, abort_flag, kWaitLimitNs)) { fail(7); break; }
                 if (ti.rows) {
-                    const CUtensorMap* mW = p.maps + 3 * (size_t)ti.pair;
+                    const CUtensorMap* mW = p.maps + kMapsPerPair * (size_t)ti.pair;
                     uint8_t* wsrc = w_ring + (size_t)ws * kWTileBytes;
-                    tma_store_2d(mW, wsrc, ti.col0, ti.row0);
-                    if (ti.wide) tma_store_2d(mW, wsrc + kWBoxBytes, ti.col0 + 64, ti.row0);
+                    store_w_tile(mW, wsrc, ti.row0, ti.col0, ti.wide, p.blk);
                     bulk_commit();
                     bulk_wait_read<0>();
                 }

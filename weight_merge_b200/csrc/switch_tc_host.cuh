@@ -42,19 +42,60 @@ inline EncodeTiledFn encode_tiled_fn() {
     return fn;
 }
 
-// W [out, in]: box 64 x 128 (cols x rows), 128B swizzle.
-// A [E, r, in]: box 64 x KP x 1, 128B swizzle (rows past r read as zero).
-// B [E, out, r]: box KP x 128 x 1, swizzle = KP*2 bytes (cols past r read as zero).
-inline bool encode_pair_maps(EncodeTiledFn enc, const PairDesc& pd, int E, int r, int kp,
-                      CUtensorMap out[3]) {
+// Blocked maps (one TMA operation per W tile and per expert's A columns)
+// need every weight's in to be a multiple of 64.
+inline bool blocked_maps_ok(const PairDesc* pairs, int64_t n) {
+    for (int64_t i = 0; i < n; ++i)
+        if (pairs[i].in % 64 != 0) return false;
+    return true;
+}
+
+// The W map alone (slot 0), plain or blocked; the re-base source W0 uses it
+// too.  Plain: W [out, in], box 64 x 128 (cols x rows).  Blocked: W viewed as
+// [in/64][out][64] (block stride 128 bytes, row stride 2*in), box 64 x 128 x 2,
+// which lands in shared memory as two 64-column halves 16 KB apart, the plain
+// layout of a wide tile.  128B swizzle either way.
+inline bool encode_w_map(EncodeTiledFn enc, const void* W, int64_t out, int64_t in, bool blk,
+                         CUtensorMap* m) {
     const cuuint32_t ones[3] = {1, 1, 1};
-    {
-        const cuuint64_t dims[2] = {(cuuint64_t)pd.in, (cuuint64_t)pd.out};
-        const cuuint64_t strides[1] = {(cuuint64_t)pd.in * 2};
-        const cuuint32_t box[2] = {64, 128};
-        if (enc(&out[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (void*)pd.W, dims, strides, box,
+    if (blk) {
+        const cuuint64_t dims[3] = {64, (cuuint64_t)out, (cuuint64_t)(in / 64)};
+        const cuuint64_t strides[2] = {(cuuint64_t)in * 2, 128};
+        const cuuint32_t box[3] = {64, 128, 2};
+        return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(W), dims, strides,
+                   box, ones, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+               CUDA_SUCCESS;
+    }
+    const cuuint64_t dims[2] = {(cuuint64_t)in, (cuuint64_t)out};
+    const cuuint64_t strides[1] = {(cuuint64_t)in * 2};
+    const cuuint32_t box[2] = {64, 128};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(W), dims, strides, box,
+               ones, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+// The kMapsPerPair maps of one (layer, target):
+// [0] W (encode_w_map);
+// [1] A [E, r, in]: box 64 x rows x 1, 128B swizzle (rows past r read as zero);
+// [2] B [E, out, r]: box KP x 128 x 1, swizzle = KP*2 bytes (cols past r read as zero);
+// [3] blocked only: A viewed as [E][in/64][r][64], box 64 x rows x 2 x 1, the
+//     two 64-column halves of one expert's slice in one operation (zeroed
+//     when plain).
+inline bool encode_pair_maps(EncodeTiledFn enc, const PairDesc& pd, int E, int r, int kp,
+                             bool blk, CUtensorMap out[kMapsPerPair]) {
+    const cuuint32_t ones[4] = {1, 1, 1, 1};
+    const cuuint32_t a_rows = (cuuint32_t)(r <= 8 ? 8 : kp);
+    if (!encode_w_map(enc, pd.W, pd.out, pd.in, blk, &out[0])) return false;
+    std::memset(&out[3], 0, sizeof(CUtensorMap));
+    if (blk) {
+        const cuuint64_t dims[4] = {64, (cuuint64_t)r, (cuuint64_t)(pd.in / 64), (cuuint64_t)E};
+        const cuuint64_t strides[3] = {(cuuint64_t)pd.in * 2, 128, (cuuint64_t)pd.in * r * 2};
+        const cuuint32_t box[4] = {64, a_rows, 2, 1};
+        if (enc(&out[3], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, (void*)pd.A, dims, strides, box,
                 ones, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return false;
     }
     {
@@ -62,7 +103,7 @@ inline bool encode_pair_maps(EncodeTiledFn enc, const PairDesc& pd, int E, int r
         const cuuint64_t strides[2] = {(cuuint64_t)pd.in * 2, (cuuint64_t)pd.in * r * 2};
         // ranks up to 8 fetch an 8-row box, other ranks a KP-row box; rows
         // past r read as zero
-        const cuuint32_t box[3] = {64, (cuuint32_t)(r <= 8 ? 8 : kp), 1};
+        const cuuint32_t box[3] = {64, a_rows, 1};
         if (enc(&out[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, (void*)pd.A, dims, strides, box,
                 ones, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                 CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
