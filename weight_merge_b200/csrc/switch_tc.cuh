@@ -189,11 +189,17 @@ __device__ __forceinline__ void epi_combine(uint32_t t_lane, const Coefs8& cf, i
     for (int ei = 0; ei < kTmemBatch; ++ei) {
         if (b0 + ei < cf.n) {
             const float c = coef_value(cf, b0 + ei);
+            const uint64_t cc = sm100::f32x2(c, c);
             float v[32];
             sm100::tmem_ld32(t_lane + 128u * ei, v);
             sm100::tmem_wait_ld();
+            // tot[i] = fma(c, v[i], tot[i]), two columns per instruction
 #pragma unroll
-            for (int i = 0; i < 32; ++i) tot[i] = __fmaf_rn(c, v[i], tot[i]);
+            for (int i = 0; i < 32; i += 2) {
+                const uint64_t r = sm100::fma_f32x2(cc, sm100::f32x2(v[i], v[i + 1]),
+                                                    sm100::f32x2(tot[i], tot[i + 1]));
+                sm100::f32x2_split(r, tot[i], tot[i + 1]);
+            }
         }
     }
 }
@@ -212,8 +218,13 @@ __device__ __forceinline__ void epi_update_row(uint8_t* rowp, int cgrp, int row,
         uint32_t wv[4] = {w[c4].x, w[c4].y, w[c4].z, w[c4].w};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const float lo = __uint_as_float(wv[j] << 16) + tot[8 * c4 + 2 * j];
-            const float hi = __uint_as_float(wv[j] & 0xffff0000u) + tot[8 * c4 + 2 * j + 1];
+            // (W_lo + tot, W_hi + tot) in one packed fp32 add
+            float lo, hi;
+            sm100::f32x2_split(
+                sm100::add_f32x2(sm100::f32x2(__uint_as_float(wv[j] << 16),
+                                              __uint_as_float(wv[j] & 0xffff0000u)),
+                                 sm100::f32x2(tot[8 * c4 + 2 * j], tot[8 * c4 + 2 * j + 1])),
+                lo, hi);
             const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
             wv[j] = *reinterpret_cast<const uint32_t*>(&b);
         }
