@@ -60,8 +60,9 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-torch-baseline", action="store_true",
                     help="skip the unfused per-weight torch addmm_ context figure")
-    ap.add_argument("--schedule", choices=["dynamic", "static"], default="dynamic",
-                    help="tile schedule of the single-CTA tensor-core kernel")
+    ap.add_argument("--schedule", choices=["auto", "dynamic", "static"], default="auto",
+                    help="tile schedule of the tensor-core kernels (auto: dynamic for the "
+                         "single-CTA kernel, static for the pair kernel)")
     ap.add_argument("--no-layerwise", action="store_true",
                     help="skip the per-layer-launch context figures (graph, per-layer routing)")
     ap.add_argument("--no-pipelined", action="store_true",
@@ -459,6 +460,17 @@ def e2e_leg(seq, prev_t, run_step, start, stop, read_routes, rebase=False):
     return ms, moving_steps(read_routes(), seq, prev_t, rebase), pe
 
 
+def effective_schedule(requested, kind):
+    """The tile schedule a launch of kernel `kind` uses under the context's
+    setting (ADAFUSE_SCHEDULE_AUTO: dynamic for the single-CTA tensor-core
+    kernel, static for the pair kernel; the other kernels are static)."""
+    if kind == 2:                      # ADAFUSE_KERNEL_TCGEN05
+        return "static" if requested == "static" else "dynamic"
+    if kind == 3:                      # ADAFUSE_KERNEL_TCGEN05_PAIR
+        return "dynamic" if requested == "dynamic" else "static"
+    return "static"
+
+
 # adafuse_get_tensor_map_layout values (ADAFUSE_MAPS_NONE, _PLAIN, _BLOCKED)
 MAP_LAYOUTS = {0: "none", 1: "plain", 2: "blocked"}
 KERNEL_NAMES = {1: "switch_mma_kernel", 2: "switch_tc_kernel", 3: "switch_tc2_kernel",
@@ -559,6 +571,7 @@ def config_leg(name, args, dev, stream, peak, peak_kind):
             "workload": workload_label(cfg, T),
             "route_source": "router" if cfg.route_mode == "router" else f"synthesised ({cfg.route_mode})",
             "tensor_maps": maps,
+            "tile_schedule": effective_schedule("auto", kind),
             "w_bytes_per_switch": w_bytes,
             "timed_switches": n,
             "switch_ms_p50": round(percentile(real, 0.5), 4),
@@ -734,8 +747,8 @@ def run_ours(args):
     sw.set_kernel({"auto": B.ADAFUSE_KERNEL_AUTO, "mma": B.ADAFUSE_KERNEL_MMA_SYNC,
                    "tc": B.ADAFUSE_KERNEL_TCGEN05, "tc2": B.ADAFUSE_KERNEL_TCGEN05_PAIR,
                    "fold": B.ADAFUSE_KERNEL_TCGEN05_FOLD}[args.kernel])
-    sw.set_schedule(B.ADAFUSE_SCHEDULE_DYNAMIC if args.schedule == "dynamic"
-                    else B.ADAFUSE_SCHEDULE_STATIC)
+    sw.set_schedule({"auto": B.ADAFUSE_SCHEDULE_AUTO, "dynamic": B.ADAFUSE_SCHEDULE_DYNAMIC,
+                     "static": B.ADAFUSE_SCHEDULE_STATIC}[args.schedule])
     # the kernel this run's switches launch (in-place top-k calls have their own choice)
     kind = sw.topk_kernel if (args.top_k != 2 and args.mode != "rebase") else sw.kernel
     maps = MAP_LAYOUTS[sw.map_layout]
@@ -975,7 +988,7 @@ def run_ours(args):
                 "parallelism": f"replicas x{world}",
                 "mode": args.mode,
                 "route_source": "router" if synth is None else f"synthesised ({cfg.route_mode})",
-                "tile_schedule": args.schedule if kind == B.ADAFUSE_KERNEL_TCGEN05 else "static",
+                "tile_schedule": effective_schedule(args.schedule, kind),
                 "tensor_maps": maps,
             },
             "switch_ms_p50": round(sw_sorted[len(sw_sorted) // 2], 4),

@@ -104,6 +104,8 @@ extern "C" {
 /* ---- tile schedules (adafuse_set_tile_schedule) ------------------------- */
 #define ADAFUSE_SCHEDULE_STATIC  0
 #define ADAFUSE_SCHEDULE_DYNAMIC 1
+#define ADAFUSE_SCHEDULE_AUTO    2  /* default: dynamic for ADAFUSE_KERNEL_TCGEN05, static
+                                       for ADAFUSE_KERNEL_TCGEN05_PAIR */
 
 /* ---- TMA tensor-map layouts (adafuse_get_tensor_map_layout) ------------- */
 #define ADAFUSE_MAPS_NONE    0  /* no tensor maps: only the mma.sync kernel runs */
@@ -236,14 +238,19 @@ ADAFUSE_API int adafuse_set_switch_kernel(adafuse_ctx* ctx, int kernel);
  * Re-base calls follow adafuse_get_switch_kernel.  Host-only. */
 ADAFUSE_API int adafuse_get_topk_switch_kernel(adafuse_ctx* ctx);
 
-/* Tile schedule of ADAFUSE_KERNEL_TCGEN05 (the other kernels always use the
- * static one).  ADAFUSE_SCHEDULE_STATIC: CTA b of the persistent grid takes
- * tiles b, b + grid, b + 2*grid, ... of the segment table.
- * ADAFUSE_SCHEDULE_DYNAMIC (default): each CTA takes its next tile from a
+/* Tile schedule of ADAFUSE_KERNEL_TCGEN05 and ADAFUSE_KERNEL_TCGEN05_PAIR
+ * (the other kernels always use the static one).  ADAFUSE_SCHEDULE_STATIC:
+ * CTA b (CTA pair b) of the persistent grid takes tiles (256 x 128 blocks)
+ * b, b + grid, b + 2*grid, ... of its table.  ADAFUSE_SCHEDULE_DYNAMIC: each
+ * CTA (the even CTA of each pair, for both) takes its next tile from a
  * context-owned ticket counter in table order, so the tiles in flight on the
  * GPU stay a compact window of the table (neighbouring W rows) however far the
  * CTAs' speeds drift apart; the launch leaves the counter at zero.
- * INVALID_ARG for any other value.  Host-only, no device work. */
+ * ADAFUSE_SCHEDULE_AUTO (default): dynamic for the single-CTA kernel, static
+ * for the pair kernel (the faster of the two for each on B200 at the 13B and
+ * Llama-3-8B shapes).  The schedule decides only which CTA takes a tile,
+ * never how a tile is computed: W is bit for bit the same.  INVALID_ARG for
+ * any other value.  Host-only, no device work. */
 ADAFUSE_API int adafuse_set_tile_schedule(adafuse_ctx* ctx, int schedule);
 
 /* Cap the persistent grid of this context's switch and re-base launches at

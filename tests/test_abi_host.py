@@ -113,6 +113,7 @@ def test_calls_on_null_context_are_invalid():
     assert L.adafuse_switch_topk_layers(None, 0, 1, None, None, None) == B.ADAFUSE_ERR_INVALID_ARG
     assert L.adafuse_rebase_topk(None, None, None) == B.ADAFUSE_ERR_INVALID_ARG
     assert L.adafuse_set_tile_schedule(None, B.ADAFUSE_SCHEDULE_DYNAMIC) == B.ADAFUSE_ERR_INVALID_ARG
+    assert L.adafuse_set_tile_schedule(None, B.ADAFUSE_SCHEDULE_AUTO) == B.ADAFUSE_ERR_INVALID_ARG
     assert L.adafuse_refresh_adapters(None, None) == B.ADAFUSE_ERR_INVALID_ARG
     assert L.adafuse_get_topk_switch_kernel(None) == B.ADAFUSE_ERR_INVALID_ARG
     assert L.adafuse_get_tensor_map_layout(None) == B.ADAFUSE_ERR_INVALID_ARG

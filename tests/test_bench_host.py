@@ -61,3 +61,15 @@ def test_route_buffer_synthesised_workloads():
     assert np.array_equal(buf4[:, 4:6].view(np.float32), gate)
     assert np.all(buf4[:, 6:].view(np.float32) == 0)
     assert bench.route_buffer(wl.CONFIGS["7b"], 16, False, "cpu") is None
+
+
+def test_effective_schedule_follows_the_auto_rule():
+    """ADAFUSE_SCHEDULE_AUTO: dynamic for the single-CTA tensor-core kernel
+    (2), static for the pair kernel (3); an explicit choice applies to both;
+    the other kernels are static."""
+    assert bench.effective_schedule("auto", 2) == "dynamic"
+    assert bench.effective_schedule("auto", 3) == "static"
+    assert bench.effective_schedule("dynamic", 3) == "dynamic"
+    assert bench.effective_schedule("static", 2) == "static"
+    for k in (1, 4):
+        assert bench.effective_schedule("dynamic", k) == "static"

@@ -340,11 +340,11 @@ def test_grid_cap_gives_the_same_w_bit_for_bit(kernel, r, cap):
     """adafuse_set_max_ctas only shrinks the persistent grid: each tile is
     computed the same way whichever CTA takes it, so a capped context and an
     uncapped one end with the same W, bit for bit, over full and layer-range
-    switches (both tile schedules of the single-CTA kernel)."""
+    switches (both tile schedules of the single-CTA and pair kernels)."""
     m1, m2 = _small_model(seed=23, r=r), _small_model(seed=23, r=r)
     s1, s2 = make_switcher(m1, kernel), make_switcher(m2, kernel)
     s2.set_max_ctas(cap)
-    if kernel == TC:
+    if kernel in (TC, TC2):
         s1.set_schedule(Bnd.ADAFUSE_SCHEDULE_STATIC)
     routes = make_routes(np.array([[0, 1], [2, 3], [1, 2]], np.int32),
                          np.array([[0.7, 0.3], [0.6, 0.4], [0.5, 0.5]], np.float32))
@@ -362,14 +362,15 @@ def test_grid_cap_gives_the_same_w_bit_for_bit(kernel, r, cap):
         s2.set_max_ctas(-1)
 
 
-@pytest.mark.parametrize("r", [8, 4, 16])
-def test_static_and_dynamic_tile_schedules_agree_bitwise(r):
-    """The schedule only decides which CTA takes a tile, never how a tile is
-    computed: a static and a dynamic context give the same W, bit for bit,
-    over repeated full and layer-range launches (the dynamic ticket counter
-    is back at zero after every launch)."""
+@pytest.mark.parametrize("kernel,r", [(TC, 8), (TC, 4), (TC, 16), (TC2, 16), (TC2, 32),
+                                      (TC2, 64)])
+def test_static_and_dynamic_tile_schedules_agree_bitwise(kernel, r):
+    """The schedule only decides which CTA (CTA pair) takes a tile, never how
+    a tile is computed: a static and a dynamic context give the same W, bit
+    for bit, over repeated full and layer-range launches (the dynamic ticket
+    counter is back at zero after every launch)."""
     m1, m2 = _small_model(seed=12, r=r), _small_model(seed=12, r=r)
-    s1, s2 = make_switcher(m1, TC), make_switcher(m2, TC)
+    s1, s2 = make_switcher(m1, kernel), make_switcher(m2, kernel)
     s1.set_schedule(Bnd.ADAFUSE_SCHEDULE_STATIC)
     s2.set_schedule(Bnd.ADAFUSE_SCHEDULE_DYNAMIC)
     routes = make_routes(np.array([[0, 1], [2, 3], [1, 2], [3, 0]], np.int32),

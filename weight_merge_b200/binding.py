@@ -31,6 +31,7 @@ ADAFUSE_KERNEL_TCGEN05_PAIR = 3
 ADAFUSE_KERNEL_TCGEN05_FOLD = 4
 ADAFUSE_SCHEDULE_STATIC = 0
 ADAFUSE_SCHEDULE_DYNAMIC = 1
+ADAFUSE_SCHEDULE_AUTO = 2
 ADAFUSE_MAPS_NONE = 0
 ADAFUSE_MAPS_PLAIN = 1
 ADAFUSE_MAPS_BLOCKED = 2

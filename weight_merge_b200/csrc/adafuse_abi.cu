@@ -47,7 +47,7 @@ struct adafuse_ctx {
     bool fold_failed = false;                // that allocation failed: the kernel is off
     float* d_logits = nullptr;               // [kMaxBatchTokens, E] batch pre-gate scratch
     unsigned long long* d_sched = nullptr;   // [2] ticket counter of the dynamic tile schedule
-    int schedule = ADAFUSE_SCHEDULE_DYNAMIC;
+    int schedule = ADAFUSE_SCHEDULE_AUTO;
     std::vector<int64_t> layer_block_begin;  // [n_layers + 1]
     int pair_clusters = 0;                   // co-resident CTA pairs (0 = not queried yet)
     int max_ctas = 0;                        // cap on a switch's persistent grid (0 = none)
@@ -265,7 +265,7 @@ cudaError_t launch_tc(adafuse_ctx* c, int64_t t0, int64_t t1, const int32_t* pre
     prm.w0_maps = c->d_w0_maps;
     prm.stall = c->stall_at;
     c->stall_at = 0;
-    prm.dyn = c->schedule == ADAFUSE_SCHEDULE_DYNAMIC ? 1 : 0;
+    prm.dyn = c->schedule != ADAFUSE_SCHEDULE_STATIC ? 1 : 0;   // AUTO: dynamic
     prm.sched = c->d_sched;
     return launch_switch_tc<KP, BBULK>(prm, c->device, switch_ctas(c), s);
 }
@@ -297,8 +297,8 @@ cudaError_t launch_tc2(adafuse_ctx* c, int64_t b0, int64_t b1, const int32_t* pr
     prm.w0_maps = c->d_w0_maps;
     prm.stall = c->stall_at;
     c->stall_at = 0;
-    prm.dyn = 0;
-    prm.sched = nullptr;
+    prm.dyn = c->schedule == ADAFUSE_SCHEDULE_DYNAMIC ? 1 : 0;   // AUTO: static
+    prm.sched = c->d_sched;
     const int cap = switch_ctas(c) / 2 > 0 ? switch_ctas(c) / 2 : 1;
     return launch_switch_tc2<KP>(prm, c->pair_clusters < cap ? c->pair_clusters : cap, s);
 }
@@ -575,7 +575,8 @@ int adafuse_get_topk_switch_kernel(adafuse_ctx* ctx) {
 
 int adafuse_set_tile_schedule(adafuse_ctx* ctx, int schedule) {
     if (ctx == nullptr) return ADAFUSE_ERR_INVALID_ARG;
-    if (schedule != ADAFUSE_SCHEDULE_STATIC && schedule != ADAFUSE_SCHEDULE_DYNAMIC)
+    if (schedule != ADAFUSE_SCHEDULE_STATIC && schedule != ADAFUSE_SCHEDULE_DYNAMIC &&
+        schedule != ADAFUSE_SCHEDULE_AUTO)
         return ADAFUSE_ERR_INVALID_ARG;
     ctx->schedule = schedule;
     return ADAFUSE_OK;

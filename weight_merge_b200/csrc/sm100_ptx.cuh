@@ -296,6 +296,16 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
     asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
 }
 
+// Asynchronous 8-byte store into the peer CTA's shared memory whose
+// completion (and visibility to the peer's waiters) is counted as 8 bytes of
+// transfer on the peer's mbarrier `bar` (both shared::cluster addresses).
+__device__ __forceinline__ void st_async_v2_cluster(uint32_t addr, uint32_t x, uint32_t y,
+                                                    uint32_t bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.u32 [%0], {%1, %2}, [%3];"
+                 ::"r"(addr), "r"(x), "r"(y), "r"(bar)
+                 : "memory");
+}
+
 // Arrive on an mbarrier of either CTA of the pair (shared::cluster address),
 // announcing `bytes` of transfers that will complete on it.
 __device__ __forceinline__ void mbar_arrive_expect_tx_cluster(uint32_t bar_cluster, uint32_t bytes) {

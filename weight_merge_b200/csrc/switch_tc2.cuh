@@ -11,7 +11,13 @@
 //     CTAs, 64 columns each, so each SM stages half of them;
 //   * the even CTA issues the MMAs; both CTAs arrive on the even CTA's "full"
 //     barrier, and their operand loads complete on it; each MMA batch's
-//     completion frees the operand stage in both CTAs.
+//     completion frees the operand stage in both CTAs;
+//   * the even CTA's W producer picks the blocks (a static stride over the
+//     table, or tickets from a per-context counter) and publishes each W
+//     stage's block entry to both CTAs: its own slot with a plain store, the
+//     odd CTA's with an 8-byte st.async that completes on the odd CTA's
+//     barrier; it reuses a stage only after both CTAs' store warps released
+//     it (the even CTA's "empty" barrier counts both).
 // Per selected expert a CTA stages 128 x r B rows + r x 64 A columns instead
 // of 128 x r + r x 128: at rank 64 that is 24 KB instead of 32 KB per tile,
 // which leaves room for a deeper operand ring next to the W ring.
@@ -49,7 +55,10 @@ struct Tc2Config {
                                        : KP == 32 ? sm100::kSwizzle64B
                                                   : sm100::kSwizzle128B;
     static constexpr uint32_t kBSbo = 8 * KP * 2;
-    static constexpr uint32_t kBarBytes = 8 * (3 * kWStages + 2 * kOpStages + 2) + 16;
+    // barriers (w_full, w_empty, epi_done, te_full per W stage; op_full,
+    // op_empty per operand stage; acc_full, acc_empty), the W stages' tile
+    // entries, tmem base + abort flag
+    static constexpr uint32_t kBarBytes = 8 * (4 * kWStages + 2 * kOpStages + 2) + 8 * kWStages + 16;
     static constexpr uint32_t kSmemBytes = 1024 + kOpBytes + kWBytes + kBarBytes;
     static_assert(kSmemBytes <= 232448, "shared memory");
     static_assert(kOpStageBytes % 1024 == 0 && kAHalfBytes % 1024 == 0, "swizzle atoms stay aligned");
@@ -92,7 +101,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc2_kernel(const TcParam
     uint64_t* acc_full = op_empty + C::kOpStages;
     uint64_t* acc_empty = acc_full + 1;            // used in the even CTA only
     uint64_t* epi_done = acc_empty + 1;            // [kWStages]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epi_done + C::kWStages);
+    uint64_t* te_full = epi_done + C::kWStages;    // [kWStages]: the stage's block entry is set
+    TileEntry* te_slot = reinterpret_cast<TileEntry*>(te_full + C::kWStages);  // [kWStages]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(te_slot + C::kWStages);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     Coefs8 cf;
@@ -104,7 +115,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc2_kernel(const TcParam
     if (cf.n == 0 && !p.rebase) return;  // identity switch (both CTAs agree)
     const int64_t n_clusters = (int64_t)cluster_count_x();
     const int64_t first = p.t_begin + (int64_t)cluster_id_x();
-    if (first >= p.t_end) return;        // both CTAs agree
+    // (the dynamic schedule needs every pair at teardown to reset its
+    // counter; the launch never has more pairs than blocks, so no pair
+    // leaves here then)
+    if (!p.dyn && first >= p.t_end) return;        // both CTAs agree
 
     const uint32_t q = cluster_ctarank();  // 0: issues the MMAs
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -112,8 +126,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc2_kernel(const TcParam
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::kWStages; ++i) {
             mbar_init(&w_full[i], 1);
-            mbar_init(&w_empty[i], 1);
+            // even CTA: its own and the odd CTA's store warp release the stage
+            mbar_init(&w_empty[i], 2);
             mbar_init(&epi_done[i], kTcEpiThreads);
+            mbar_init(&te_full[i], 1);
         }
         for (int i = 0; i < C::kOpStages; ++i) {
             // one arrival (with its own bytes) from each CTA per use: the even
@@ -148,20 +164,47 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc2_kernel(const TcParam
 
     if (warp == 0) {
         // ---------------- W producer: this CTA's tiles into the W ring ----
+        // The even CTA's picks the blocks for both CTAs (see the file head);
+        // the odd CTA's takes them from its tile-entry slots.
         if (lane == 0) {
             int ws = 0;
             uint32_t wph = 0;
             uint32_t last_pair = 0xffffffffu;
-            TileEntry te_next = fetch_tile(p.tiles, first, p.t_end);
-            for (int64_t t = first; t < p.t_end && !*abort_flag; t += n_clusters) {
-                const PairTile ti = decode_pair_tile(te_next, q);
-                te_next = fetch_tile(p.tiles, t + n_clusters, p.t_end);
+            const uint32_t peer_te_full = cluster_addr(te_full, 1);
+            const uint32_t peer_te_slot = cluster_addr(te_slot, 1);
+            auto next_block = [&](int64_t t) -> int64_t {
+                if (t >= p.t_end) return t;
+                return p.dyn ? p.t_begin + (int64_t)atomicAdd(p.sched, 1ull) : t + n_clusters;
+            };
+            int64_t t = 0, tn = 0;
+            TileEntry te = make_uint2(0u, 0u), te_n = te;
+            if (q == 0) {
+                t = p.dyn ? next_block(p.t_begin) : first;
+                te = fetch_tile(p.tiles, t, p.t_end);
+            }
+            while (!*abort_flag) {
+                if (q == 0) {
+                    tn = next_block(t);
+                    te_n = fetch_tile(p.tiles, tn, p.t_end);
+                    if (!mbar_wait_bounded(&w_empty[ws], wph ^ 1, abort_flag, kWaitLimitNs)) { fail(1); break; }
+                    const TileEntry pub = t >= p.t_end ? make_uint2(kTileEndX, kTileEndX) : te;
+                    te_slot[ws] = pub;
+                    mbar_arrive(&te_full[ws]);
+                    const uint32_t pf = peer_te_full + 8u * (uint32_t)ws;
+                    mbar_arrive_expect_tx_cluster(pf, 8u);
+                    st_async_v2_cluster(peer_te_slot + 8u * (uint32_t)ws, pub.x, pub.y, pf);
+                    if (t >= p.t_end) break;
+                } else {
+                    if (!mbar_wait_bounded(&te_full[ws], wph, abort_flag, kWaitLimitNs)) { fail(1); break; }
+                    te = te_slot[ws];
+                    if (te.x == kTileEndX) break;
+                }
+                const PairTile ti = decode_pair_tile(te, q);
                 const CUtensorMap* mW = p.rebase ? p.w0_maps + ti.pair : p.maps + kMapsPerPair * (size_t)ti.pair;
                 if (ti.pair != last_pair) {
                     tensormap_acquire(mW);
                     last_pair = ti.pair;
                 }
-                if (!mbar_wait_bounded(&w_empty[ws], wph ^ 1, abort_flag, kWaitLimitNs)) { fail(1); break; }
                 uint8_t* wdst = w_ring + (size_t)ws * kWTileBytes;
                 if (ti.rows) {
                     mbar_arrive_expect_tx(&w_full[ws], w_tile_bytes(p.blk, ti.wide));
@@ -171,9 +214,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc2_kernel(const TcParam
                     mbar_arrive(&w_full[ws]);
                 }
                 if (++ws == C::kWStages) { ws = 0; wph ^= 1; }
-                if (t + n_clusters < p.t_end && (te_next.x & kTile2PairMask) != ti.pair) {
-                    const uint32_t np = te_next.x & kTile2PairMask;
-                    tensormap_prefetch(p.rebase ? p.w0_maps + np : p.maps + kMapsPerPair * (size_t)np);
+                if (q == 0) {
+                    if (tn < p.t_end && (te_n.x & kTile2PairMask) != ti.pair) {
+                        const uint32_t np = te_n.x & kTile2PairMask;
+                        tensormap_prefetch(p.rebase ? p.w0_maps + np : p.maps + kMapsPerPair * (size_t)np);
+                    }
+                    t = tn;
+                    te = te_n;
                 }
             }
         }
@@ -183,14 +230,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc2_kernel(const TcParam
         // even CTA's full barrier ----
         if (lane == 0) {
             const uint32_t full0 = cluster_addr(op_full, 0);
-            int os = 0;
-            uint32_t oph = 0;
+            int os = 0, ts = 0;
+            uint32_t oph = 0, tph = 0;
             uint32_t last_pair = 0xffffffffu;
             bool ok = true;
-            TileEntry te_next = fetch_tile(p.tiles, first, p.t_end);
-            for (int64_t t = first; t < p.t_end && !*abort_flag; t += n_clusters) {
-                const PairTile ti = decode_pair_tile(te_next, q);
-                te_next = fetch_tile(p.tiles, t + n_clusters, p.t_end);
+            int tile_no = 0;   // blocks this pair has taken (for the stall hook)
+            while (!*abort_flag) {
+                if (!mbar_wait_bounded(&te_full[ts], tph, abort_flag, kWaitLimitNs)) { ok = false; break; }
+                const TileEntry te = te_slot[ts];
+                if (++ts == C::kWStages) { ts = 0; tph ^= 1; }
+                if (te.x == kTileEndX) break;
+                const bool stall_here = ++tile_no == p.stall;
+                const PairTile ti = decode_pair_tile(te, q);
                 const CUtensorMap* mA = p.maps + kMapsPerPair * (size_t)ti.pair + 1;
                 const CUtensorMap* mB = mA + 1;
                 if (ti.pair != last_pair) {
@@ -208,19 +259,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc2_kernel(const TcParam
                     uint8_t* b_dst = a_dst + C::kAHalfBytes;
                     const uint32_t full = full0 + 8u * (uint32_t)os;
                     mbar_arrive_expect_tx_cluster(
-                        full, bytes + (q == 0 && ei == 0 && (t - first) / n_clusters + 1 == p.stall
-                                           ? kStallBytes : 0u));
+                        full, bytes + (q == 0 && ei == 0 && stall_here ? kStallBytes : 0u));
                     if (ti.rows) tma_load_3d_pair(b_dst, mB, 0, ti.row0, e, full);
                     if (load_a) tma_load_3d_pair(a_dst, mA, ti.col0 + 64 * (int)q, 0, e, full);
                     if (++os == C::kOpStages) { os = 0; oph ^= 1; }
                 }
-                if (!ok) { fail(2); break; }
-                if (t + n_clusters < p.t_end && (te_next.x & kTile2PairMask) != ti.pair) {
-                    const CUtensorMap* nm = p.maps + kMapsPerPair * (size_t)(te_next.x & kTile2PairMask);
-                    tensormap_prefetch(nm + 1);
-                    tensormap_prefetch(nm + 2);
-                }
+                if (!ok) break;
             }
+            if (!ok) fail(2);
             // every stage filled here is released by an MMA completion that
             // arrives on this CTA's barrier: see the last ones land
             for (int j = 0; ok && !*abort_flag && j < C::kOpStages; ++j) {
@@ -232,11 +278,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc2_kernel(const TcParam
         // ---------------- MMA issuer (even CTA) ----------------
         if (lane == 0 && q == 0) {
             constexpr uint32_t idesc = instr_desc_bf16(kBlockRows, 128, /*B MN-major*/ 1);
-            int os = 0;
-            uint32_t oph = 0, aph = 0;
+            int os = 0, ts = 0;
+            uint32_t oph = 0, aph = 0, tph = 0;
             const int nb = tmem_batches(cf);
             bool ok = true;
-            for (int64_t t = first; t < p.t_end && ok && !*abort_flag; t += n_clusters) {
+            while (ok && !*abort_flag) {
+                if (!mbar_wait_bounded(&te_full[ts], tph, abort_flag, kWaitLimitNs)) { fail(9); break; }
+                const bool end = te_slot[ts].x == kTileEndX;
+                if (++ts == C::kWStages) { ts = 0; tph ^= 1; }
+                if (end) break;
 #pragma unroll 1
               for (int b0 = 0; b0 < nb * kTmemBatch && ok; b0 += kTmemBatch) {
                 if (!mbar_wait_bounded(acc_empty, aph ^ 1, abort_flag, kWaitLimitNs)) { fail(3); ok = false; break; }
@@ -272,10 +322,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc2_kernel(const TcParam
         if (lane == 0) {
             int ws = 0;
             uint32_t wph = 0;
-            TileEntry te_next = fetch_tile(p.tiles, first, p.t_end);
-            for (int64_t t = first; t < p.t_end && !*abort_flag; t += n_clusters) {
-                const PairTile ti = decode_pair_tile(te_next, q);
-                te_next = fetch_tile(p.tiles, t + n_clusters, p.t_end);
+            // the stage is released on the even CTA's "empty" barrier (it
+            // counts both CTAs' store warps)
+            const uint32_t w_empty0 = cluster_addr(w_empty, 0);
+            while (!*abort_flag) {
+                if (!mbar_wait_bounded(&te_full[ws], wph, abort_flag, kWaitLimitNs)) { fail(10); break; }
+                const TileEntry te = te_slot[ws];
+                if (te.x == kTileEndX) break;
+                const PairTile ti = decode_pair_tile(te, q);
                 if (!mbar_wait_bounded(&epi_done[ws], wph, abort_flag, kWaitLimitNs)) { fail(7); break; }
                 if (ti.rows) {
                     const CUtensorMap* mW = p.maps + kMapsPerPair * (size_t)ti.pair;
@@ -284,7 +338,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc2_kernel(const TcParam
                     bulk_commit();
                     bulk_wait_read<0>();
                 }
-                mbar_arrive(&w_empty[ws]);
+                mbar_arrive_cluster(w_empty0 + 8u * (uint32_t)ws);
                 if (++ws == C::kWStages) { ws = 0; wph ^= 1; }
             }
             bulk_wait<0>();
@@ -301,8 +355,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc2_kernel(const TcParam
         const int nb = tmem_batches(cf);
         int ws = 0;
         uint32_t wph = 0, aph = 0;
-        for (int64_t t = first; t < p.t_end; t += n_clusters) {
+        for (;;) {
             if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+            {
+                const bool ok = mbar_wait_bounded(&te_full[ws], wph, abort_flag, kWaitLimitNs);
+                if (!__all_sync(0xffffffffu, ok)) { fail(11); break; }
+                if (te_slot[ws].x == kTileEndX) break;   // the same for every thread
+            }
             // one TMEM batch of up to four experts at a time
             float tot[32];
 #pragma unroll
@@ -344,6 +403,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc2_kernel(const TcParam
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc_pair(tmem_base, 512);
+    }
+    // dynamic schedule: every pair has taken its last ticket by now; the last
+    // one to get here leaves the counter at zero for the next launch
+    if (p.dyn && q == 0 && threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(p.sched + 1, 1ull) == (unsigned long long)n_clusters - 1) {
+            atomicExch(p.sched, 0ull);
+            atomicExch(p.sched + 1, 0ull);
+        }
     }
 }
 
