@@ -200,25 +200,40 @@ pregate_kernel(const float* __restrict__ h, int64_t T, int64_t d, const float* _
 // -- so both kernels give the same bits for the same token, and the launch
 // may pick either by batch size without changing any route.
 //
-// What changes is who does the work.  One warp owns a group of kGroupTokens
-// tokens and walks the eight virtual warps itself: per virtual warp its lanes
-// load the group's h chunks (the next virtual warp's loads are issued before
-// this one's arithmetic), read Wr's rows from shared memory (staged once per
-// CTA, shared by the group's tokens), and finish the virtual warp's sums with
-// a reduce-scatter over the same lane pairs as the xor tree (5 rounds, 31
-// shuffles for 32 (token, expert) sums), after which lane L holds token L / 8,
-// expert L % 8.  No warp waits for another after the prologue; four lanes run
-// the four tokens' top-k tails side by side.
+// What changes is who does the work.  A pair of warps owns a group of
+// kGroupTokens tokens: the even warp walks virtual warps 0..3, the odd warp
+// 4..7.  Per virtual warp and chunk index m a warp's lanes load the group's h
+// chunks (two such steps ahead of the arithmetic, in a ring of four register
+// slots), read Wr's rows from shared memory (staged once per CTA, shared by
+// the group's tokens) and accumulate; a reduce-scatter over the same lane
+// pairs as the xor tree (5 rounds, 31 shuffles for 32 (token, expert) sums)
+// then leaves lane L with token L / 8, expert L % 8 of that virtual warp.  The
+// even warp adds its four sums in order and hands the partial sum to the odd
+// warp through shared memory (a 64-thread named barrier per pair, buffers
+// alternating by group), which adds its own four in order: the same eight
+// additions as one warp walking all eight.  Four lanes of the odd warp then
+// run the four tokens' top-k tails side by side.
+// bar.sync on barrier `id` for `nthreads` threads (whole warps) of the CTA;
+// orders their shared-memory accesses like __syncthreads does for all.
+__device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 constexpr int kGroupTokens = 4;
-constexpr int kGroupThreads = 256;
+constexpr int kGroupThreads = 512;                // 8 warp pairs
+constexpr int kGroupPairs = kGroupThreads / 64;
 constexpr int kGroupMaxChunks = 4;                 // d <= 256 * 4 * 4 = 4096
 constexpr int64_t kGroupMinTokens = 64;           // smaller batches: pregate_kernel
 
-__host__ __device__ constexpr size_t group_smem_bytes(int64_t d) {
+__host__ __device__ constexpr size_t group_wr_bytes(int64_t d) {
     // Wr: one 4-row chunk (8 experts) per 9 float4 slots -- 8 of data, 1 of
     // padding, so lanes reading their own chunks 144 bytes apart hit
     // distinct bank groups
     return (size_t)(d / 4) * 9 * 16;
+}
+__host__ __device__ constexpr size_t group_smem_bytes(int64_t d) {
+    // + the pairs' partial sums, two buffers of 32 lanes each
+    return group_wr_bytes(d) + (size_t)kGroupPairs * 2 * 32 * sizeof(float);
 }
 
 template <int NCH>
@@ -227,35 +242,51 @@ pregate_group_kernel(const float* __restrict__ h, int64_t T, int64_t d,
                      const float* __restrict__ Wr, int E, int k, int slots,
                      int32_t* __restrict__ route, float* __restrict__ logits) {
     extern __shared__ __align__(128) float4 wr_s[];
+    float* zpart_s = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(wr_s) + group_wr_bytes(d));
     const int64_t nchunk = d >> 2;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int pair = warp >> 1, half = warp & 1;
     constexpr int TPB = kGroupTokens;
+    constexpr int kSteps = 4 * NCH;   // (virtual warp, chunk index) steps per warp and group
     const int64_t ngroups = (T + TPB - 1) / TPB;
     // groups go round the CTAs first, so every SM gets a share of a batch
-    const int64_t g_first = blockIdx.x + (int64_t)warp * gridDim.x;
-    const int64_t g_step = (int64_t)gridDim.x * (kGroupThreads / 32);
-    // h chunks of one virtual warp for a group's tokens (zero past T)
-    auto load_h = [&](int64_t t0, int vw, float4 (&hv)[TPB][NCH]) {
+    const int64_t g_first = blockIdx.x + (int64_t)pair * gridDim.x;
+    const int64_t g_step = (int64_t)gridDim.x * kGroupPairs;
+    // step s of this warp in group g: virtual warp 4 * half + s / NCH, chunk
+    // index s % NCH; the group's h chunks for it (zero past d or T).  Groups
+    // of 4 whole tokens with d = 1024 * NCH (every chunk inside d) take the
+    // unchecked loads.  d <= 4096 here, so token offsets fit 32 bits.
+    const bool d_full = nchunk == 256 * NCH;
+    const int nch32 = (int)nchunk;
+    const int lane_c = 128 * half + lane;            // chunk of step 0 (vw = 4 * half)
+    auto group_ptr = [&](int64_t g) {
+        return reinterpret_cast<const float4*>(h) + g * TPB * nchunk + lane_c;
+    };
+    auto load_step = [&](const float4* gp, int64_t g, int s, float4 (&hv)[TPB]) {
+        const int off = 32 * (s / NCH) + 256 * (s % NCH);
+        const int c = lane_c + off;
+        const int64_t t0 = g * TPB;
+        if (d_full && t0 + TPB <= T) {
 #pragma unroll
-        for (int m = 0; m < NCH; ++m) {
-            const int64_t c = 32 * vw + lane + 256 * m;
+            for (int tt = 0; tt < TPB; ++tt) hv[tt] = __ldcs(gp + off + tt * nch32);
+        } else {
 #pragma unroll
             for (int tt = 0; tt < TPB; ++tt)
-                hv[tt][m] = (c < nchunk && t0 + tt < T)
-                                ? __ldcs(reinterpret_cast<const float4*>(h + (t0 + tt) * d) + c)
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
+                hv[tt] = (c < nch32 && t0 + tt < T) ? __ldcs(gp + off + tt * nch32)
+                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
         }
     };
-    float4 ha[TPB][NCH], hb[TPB][NCH];
+    float4 ring[4][TPB];   // step s in slot s % 4 (kSteps is a multiple of 4)
     // the first group's first loads go out before Wr is staged, so the two
     // latencies overlap
-    if (g_first < ngroups) load_h(g_first * TPB, 0, ha);
+    load_step(group_ptr(g_first), g_first, 0, ring[0]);
+    load_step(group_ptr(g_first), g_first, 1, ring[1]);
 
     // ---- Wr into shared memory: chunk c's rows 4c..4c+3 (experts 0..7, zero
     // past E) as float4 slots c * 9 + 2 * q + (e / 4), kStageBatch loads in
     // flight per thread before their stores
     {
-        constexpr int kStageBatch = 16;
+        constexpr int kStageBatch = 8;
         const bool vec = E == 8 && (reinterpret_cast<uintptr_t>(Wr) & 15u) == 0;
         const int64_t total = nchunk * 8;
         for (int64_t i0 = threadIdx.x; i0 < total; i0 += kStageBatch * kGroupThreads) {
@@ -289,76 +320,103 @@ pregate_group_kernel(const float* __restrict__ h, int64_t T, int64_t d,
 
     const bool b16 = (lane & 16) != 0, b8 = (lane & 8) != 0, b4 = (lane & 4) != 0,
                b2 = (lane & 2) != 0, b1 = (lane & 1) != 0;
-    for (int64_t g = g_first; g < ngroups; g += g_step) {
-        const int64_t t0 = g * TPB;
-        if (g != g_first) load_h(t0, 0, ha);
-        float zsum = 0.f;   // lane L: the in-order sum for token L / 8, expert L % 8
+    int parity = 0;
+    for (int64_t g = g_first; g < ngroups; g += g_step, parity ^= 1) {
+        const float4* gp = group_ptr(g);
+        const float4* gp_next = group_ptr(g + g_step);
+        float zs[4];   // lane L: this warp's four virtual-warp sums for token L / 8, expert L % 8
+        // acc2[tt][p]: experts 2p and 2p + 1 of token tt as a packed fp32
+        // pair; fma.rn.f32x2 rounds each lane as fma.rn.f32 does, so every
+        // (token, expert) sum takes the FMA sequence of pregate_kernel
+        uint64_t acc2[TPB][4];
 #pragma unroll
-        for (int vw = 0; vw < 8; ++vw) {
-            float4 (&hc)[TPB][NCH] = (vw & 1) ? hb : ha;
-            float4 (&hn)[TPB][NCH] = (vw & 1) ? ha : hb;
-            if (vw + 1 < 8) load_h(t0, vw + 1, hn);
-            float acc[TPB][8];
+        for (int s = 0; s < kSteps; ++s) {
+            const int m = s % NCH;
+            const int vw = 4 * half + s / NCH;
+            // two steps ahead: this group's step s + 2, or the next group's
+            if (s + 2 < kSteps)
+                load_step(gp, g, s + 2, ring[(s + 2) & 3]);
+            else
+                load_step(gp_next, g + g_step, s + 2 - kSteps, ring[(s + 2) & 3]);
+            if (m == 0) {
 #pragma unroll
-            for (int tt = 0; tt < TPB; ++tt)
+                for (int tt = 0; tt < TPB; ++tt)
 #pragma unroll
-                for (int e = 0; e < 8; ++e) acc[tt][e] = 0.f;
+                    for (int pe = 0; pe < 4; ++pe) acc2[tt][pe] = 0ull;
+            }
+            const int c = 32 * vw + lane + 256 * m;
+            if (d_full || c < nch32) {
 #pragma unroll
-            for (int m = 0; m < NCH; ++m) {
-                const int64_t c = 32 * vw + lane + 256 * m;
-                if (c < nchunk) {
-                    float w[4][8];
+                for (int q = 0; q < 4; ++q) {
+                    const float4 wa = wr_s[c * 9 + 2 * q], wb = wr_s[c * 9 + 2 * q + 1];
+                    const uint64_t w2[4] = {sm100::f32x2(wa.x, wa.y), sm100::f32x2(wa.z, wa.w),
+                                            sm100::f32x2(wb.x, wb.y), sm100::f32x2(wb.z, wb.w)};
 #pragma unroll
-                    for (int f = 0; f < 8; ++f) {
-                        const float4 v = wr_s[c * 9 + f];
-                        w[f >> 1][(f & 1) * 4 + 0] = v.x;
-                        w[f >> 1][(f & 1) * 4 + 1] = v.y;
-                        w[f >> 1][(f & 1) * 4 + 2] = v.z;
-                        w[f >> 1][(f & 1) * 4 + 3] = v.w;
+                    for (int tt = 0; tt < TPB; ++tt) {
+                        const float4 x4 = ring[s & 3][tt];
+                        const float x = q == 0 ? x4.x : q == 1 ? x4.y : q == 2 ? x4.z : x4.w;
+                        const uint64_t xx = sm100::f32x2(x, x);
+#pragma unroll
+                        for (int pe = 0; pe < 4; ++pe)
+                            acc2[tt][pe] = sm100::fma_f32x2(xx, w2[pe], acc2[tt][pe]);
                     }
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-#pragma unroll
-                        for (int e = 0; e < 8; ++e)
-#pragma unroll
-                            for (int tt = 0; tt < TPB; ++tt) {
-                                const float4 x4 = hc[tt][m];
-                                const float x = q == 0 ? x4.x : q == 1 ? x4.y : q == 2 ? x4.z : x4.w;
-                                acc[tt][e] = __fmaf_rn(x, w[q][e], acc[tt][e]);
-                            }
                 }
             }
-            // the virtual warp's 32 sums (value index tt * 8 + e) by
-            // reduce-scatter: each round a lane keeps the half of its values
-            // its lane bit selects and adds its partner's copies of them, the
-            // pairs the xor tree adds; lane L ends with value L
-            float r16[16];
+            if (m == NCH - 1) {
+                float acc[TPB][8];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const float lo = acc[i >> 3][i & 7], hi = acc[(16 + i) >> 3][(16 + i) & 7];
-                r16[i] = (b16 ? hi : lo) + __shfl_xor_sync(0xffffffffu, b16 ? lo : hi, 16);
+                for (int tt = 0; tt < TPB; ++tt)
+#pragma unroll
+                    for (int pe = 0; pe < 4; ++pe)
+                        sm100::f32x2_split(acc2[tt][pe], acc[tt][2 * pe], acc[tt][2 * pe + 1]);
+                // the virtual warp's 32 sums (value index tt * 8 + e) by
+                // reduce-scatter: each round a lane keeps the half of its
+                // values its lane bit selects and adds its partner's copies of
+                // them, the pairs the xor tree adds; lane L ends with value L
+                float r16[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float lo = acc[i >> 3][i & 7], hi = acc[(16 + i) >> 3][(16 + i) & 7];
+                    r16[i] = (b16 ? hi : lo) + __shfl_xor_sync(0xffffffffu, b16 ? lo : hi, 16);
+                }
+                float r8[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    r8[i] = (b8 ? r16[8 + i] : r16[i]) +
+                            __shfl_xor_sync(0xffffffffu, b8 ? r16[i] : r16[8 + i], 8);
+                float r4[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    r4[i] = (b4 ? r8[4 + i] : r8[i]) +
+                            __shfl_xor_sync(0xffffffffu, b4 ? r8[i] : r8[4 + i], 4);
+                float r2[2];
+#pragma unroll
+                for (int i = 0; i < 2; ++i)
+                    r2[i] = (b2 ? r4[2 + i] : r4[i]) +
+                            __shfl_xor_sync(0xffffffffu, b2 ? r4[i] : r4[2 + i], 2);
+                zs[s / NCH] = (b1 ? r2[1] : r2[0]) +
+                              __shfl_xor_sync(0xffffffffu, b1 ? r2[0] : r2[1], 1);
             }
-            float r8[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                r8[i] = (b8 ? r16[8 + i] : r16[i]) +
-                        __shfl_xor_sync(0xffffffffu, b8 ? r16[i] : r16[8 + i], 8);
-            float r4[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                r4[i] = (b4 ? r8[4 + i] : r8[i]) +
-                        __shfl_xor_sync(0xffffffffu, b4 ? r8[i] : r8[4 + i], 4);
-            float r2[2];
-#pragma unroll
-            for (int i = 0; i < 2; ++i)
-                r2[i] = (b2 ? r4[2 + i] : r4[i]) +
-                        __shfl_xor_sync(0xffffffffu, b2 ? r4[i] : r4[2 + i], 2);
-            const float r1 = (b1 ? r2[1] : r2[0]) + __shfl_xor_sync(0xffffffffu, b1 ? r2[0] : r2[1], 1);
-            zsum = vw == 0 ? r1 : zsum + r1;
         }
+        // the eight virtual-warp sums in order: virtual warps 0..3 here (even
+        // warp), then 4..7 on top of them (odd warp)
+        float* buf = zpart_s + (pair * 2 + parity) * 32;
+        float zsum;
+        if (half == 0) {
+            zsum = zs[0];
+#pragma unroll
+            for (int i = 1; i < 4; ++i) zsum = zsum + zs[i];
+            buf[lane] = zsum;
+            named_barrier_sync(1 + pair, 64);
+            continue;
+        }
+        named_barrier_sync(1 + pair, 64);
+        zsum = buf[lane];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) zsum = zsum + zs[i];
         // ---- the group's decisions: lane 8 * tt gathers token tt's logits
         const int tt = lane >> 3, e = lane & 7;
-        const int64_t t = t0 + tt;
+        const int64_t t = g * TPB + tt;
         if (logits != nullptr) {
             if (t < T && e < E) logits[t * E + e] = zsum;
         } else {
@@ -369,6 +427,7 @@ pregate_group_kernel(const float* __restrict__ h, int64_t T, int64_t d,
         }
     }
 }
+
 
 // ---------------------------------------------------------------------------
 // One routing decision for a decode batch: the kernels above, given a logits
