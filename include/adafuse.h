@@ -439,8 +439,9 @@ ADAFUSE_API int adafuse_segment_table(const adafuse_desc* desc, int32_t* entries
  * call returns), so ALL calls share it: two calls whose work overlaps on the
  * GPU (different streams, or threads without ordering) race and may switch
  * the wrong weights.  Calls on one stream are ordered and safe.  The first
- * call on each device also looks up the array's device address (once per
- * device); make that first call before any stream capture.
+ * call on each device also looks up the array's device address
+ * (cudaGetSymbolAddress, once per device, under a host mutex that guards
+ * only that lookup).
  *
  * Arguments: desc as for adafuse_create (host memory, read during the call
  * only; its device pointers must stay valid until the switch completes);

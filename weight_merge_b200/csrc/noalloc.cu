@@ -17,8 +17,7 @@
 // whose work overlaps on the GPU (different streams, or different host
 // threads without ordering) race on it.  Calls on one stream are ordered and
 // safe.  The first call on a device looks up the array's device address
-// (cudaGetSymbolAddress) once for that device; make that first call before
-// any stream capture.
+// (cudaGetSymbolAddress) once for that device.
 #include <cuda_runtime.h>
 
 #include <cmath>
