@@ -140,6 +140,29 @@ def test_pregate_matches_oracle(T, d, E):
         assert np.all(got[:, 1] == -1)
 
 
+@pytest.mark.parametrize("T,d,E", [(65, 12, 3), (131, 1028, 5), (1027, 2948, 8), (66, 3072, 8),
+                                   (257, 4092, 7), (64, 1024, 2)])
+def test_batch_router_matches_the_one_token_router_bit_for_bit(T, d, E):
+    """The batch kernel (a warp pair per 4-token group, the odd warp adding
+    its four virtual-warp sums on top of the even warp's) against one-token
+    launches of the decode kernel, for every token: partial last groups,
+    every chunk count 1..4, chunks past d, fewer than 8 experts.  Routes must
+    agree bit for bit (indices and gate bits)."""
+    cfg = wl.custom("p", 1, [("q", 8, 8)], n_experts=E, rank=8, alpha=16, n_tokens=T, d=d)
+    sw = make_switcher(wl.make_model(cfg, device="cuda"))
+    g = torch.Generator(device="cuda").manual_seed(T + d + E)
+    h = torch.randn((T, d), generator=g, device="cuda")
+    Wr = torch.randn((d, E), generator=g, device="cuda") * 0.05
+    batch = torch.zeros((T, 4), dtype=torch.int32, device="cuda")
+    sw.pregate(h, Wr, batch, stream())
+    single = torch.zeros((T, 4), dtype=torch.int32, device="cuda")
+    for t in range(T):
+        sw.pregate(h[t:t + 1], Wr, single[t:t + 1], stream())
+    torch.cuda.synchronize()
+    assert torch.equal(batch, single)
+    sw.close()
+
+
 @pytest.mark.parametrize("E", [8, 16])
 def test_pregate_route_does_not_depend_on_batch_size(E):
     """A token's route is bitwise the same whether it is gated alone or inside
