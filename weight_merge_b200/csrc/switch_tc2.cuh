@@ -164,8 +164,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) switch_tc2_kernel(const TcParam
 
     if (warp == 0) {
         // ---------------- W producer: this CTA's tiles into the W ring ----
-        // The even CTA's picks the blocks for both CTAs (see the file head);
-        // the odd CTA's takes them from its tile-entry slots.
+        // The even CTA's producer picks the blocks for both CTAs (see the file
+        // head); the odd CTA's producer takes them from its tile-entry slots.
         if (lane == 0) {
             int ws = 0;
             uint32_t wph = 0;
