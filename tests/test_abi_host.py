@@ -126,3 +126,46 @@ def test_segment_table_capacity_checked():
     buf = (ctypes.c_int32 * 8)()
     assert B.lib().adafuse_segment_table(ctypes.byref(d), buf, 2, ctypes.byref(n)) == B.ADAFUSE_ERR_INVALID_ARG
     assert n.value == 4
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    """include/adafuse.h compiles as C99 with warnings as errors, and a C
+    program that takes the address of every declared entry point links
+    against the library and runs its host-only calls (no GPU work)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not found")
+    syms = declared_symbols()
+    lib = B.library_path()
+    src = tmp_path / "abi_check.c"
+    src.write_text(
+        '#include <stdio.h>\n#include <string.h>\n#include "adafuse.h"\n'
+        "int main(void) {\n"
+        "    const void* fns[] = {\n" + "".join(f"        (const void*)&{s},\n" for s in syms) +
+        "    };\n"
+        "    adafuse_ctx* ctx = 0;\n"
+        "    int64_t n = -1;\n"
+        "    adafuse_target tg;\n"
+        "    adafuse_desc d;\n"
+        "    memset(&tg, 0, sizeof tg);\n"
+        "    memset(&d, 0, sizeof d);\n"
+        "    tg.out = 256; tg.in = 384;\n"
+        "    d.n_layers = 1; d.n_targets = 1; d.n_experts = 2; d.rank = 8; d.alpha = 16.0f;\n"
+        "    d.targets = &tg;\n"
+        "    if (fns[0] == 0) return 1;\n"
+        "    if (adafuse_tile_size() != 128) return 2;\n"
+        "    if (adafuse_create(&ctx, 0, 0) != ADAFUSE_ERR_INVALID_ARG) return 3;\n"
+        "    if (adafuse_segment_table(&d, 0, 0, &n) != ADAFUSE_OK || n != 6) return 4;\n"
+        "    printf(\"%s\\n\", adafuse_strerror(ADAFUSE_ERR_INVALID_ARG));\n"
+        "    return 0;\n"
+        "}\n")
+    exe = tmp_path / "abi_check"
+    cmd = [gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+           str(src), "-o", str(exe), lib, "-Wl,-rpath," + os.path.dirname(lib)]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
+    assert r.stdout.strip()
