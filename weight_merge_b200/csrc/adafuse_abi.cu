@@ -245,12 +245,14 @@ cudaError_t copy_padded_b(const adafuse_ctx* c, cudaStream_t s) {
 
 int kp_class(int r) { return r <= 8 ? 8 : r <= 16 ? 16 : r <= 32 ? 32 : 64; }
 
-template <int KP, bool BBULK>
-cudaError_t launch_tc(adafuse_ctx* c, int64_t t0, int64_t t1, const int32_t* prev,
-                      const int32_t* cur, int slots, cudaStream_t s, bool rebase) {
+// The parameters of one tensor-core launch over entries [t0, t1) of `tiles`
+// (the tile table, or the block table for the pair kernel).  Consumes the
+// pending stall-hook request, so it applies to exactly one launch.
+TcParams tc_params(adafuse_ctx* c, const TileEntry* tiles, int64_t t0, int64_t t1,
+                   const int32_t* prev, const int32_t* cur, int slots, bool rebase, bool dyn) {
     TcParams prm;
     prm.pairs = c->d_pairs;
-    prm.tiles = c->d_tiles;
+    prm.tiles = tiles;
     prm.maps = c->d_maps;
     prm.blk = c->blk ? 1 : 0;
     prm.t_begin = t0;
@@ -265,8 +267,17 @@ cudaError_t launch_tc(adafuse_ctx* c, int64_t t0, int64_t t1, const int32_t* pre
     prm.w0_maps = c->d_w0_maps;
     prm.stall = c->stall_at;
     c->stall_at = 0;
-    prm.dyn = c->schedule != ADAFUSE_SCHEDULE_STATIC ? 1 : 0;   // AUTO: dynamic
-    prm.sched = c->d_sched;
+    prm.dyn = dyn ? 1 : 0;
+    prm.sched = dyn ? c->d_sched : nullptr;
+    return prm;
+}
+
+template <int KP, bool BBULK>
+cudaError_t launch_tc(adafuse_ctx* c, int64_t t0, int64_t t1, const int32_t* prev,
+                      const int32_t* cur, int slots, cudaStream_t s, bool rebase) {
+    // AUTO schedule: dynamic for this kernel
+    const TcParams prm = tc_params(c, c->d_tiles, t0, t1, prev, cur, slots, rebase,
+                                   c->schedule != ADAFUSE_SCHEDULE_STATIC);
     return launch_switch_tc<KP, BBULK>(prm, c->device, switch_ctas(c), s);
 }
 
@@ -280,25 +291,9 @@ cudaError_t launch_tc2(adafuse_ctx* c, int64_t b0, int64_t b1, const int32_t* pr
             return e;
         }
     }
-    TcParams prm;
-    prm.pairs = c->d_pairs;
-    prm.tiles = c->d_blocks;
-    prm.maps = c->d_maps;
-    prm.blk = c->blk ? 1 : 0;
-    prm.t_begin = b0;
-    prm.t_end = b1;
-    prm.prev = prev;
-    prm.cur = cur;
-    prm.slots = slots;
-    prm.E = c->n_experts;
-    prm.s = c->scale;
-    prm.status = c->d_status;
-    prm.rebase = rebase ? 1 : 0;
-    prm.w0_maps = c->d_w0_maps;
-    prm.stall = c->stall_at;
-    c->stall_at = 0;
-    prm.dyn = c->schedule == ADAFUSE_SCHEDULE_DYNAMIC ? 1 : 0;   // AUTO: static
-    prm.sched = c->d_sched;
+    // AUTO schedule: static for the pair kernel
+    const TcParams prm = tc_params(c, c->d_blocks, b0, b1, prev, cur, slots, rebase,
+                                   c->schedule == ADAFUSE_SCHEDULE_DYNAMIC);
     const int cap = switch_ctas(c) / 2 > 0 ? switch_ctas(c) / 2 : 1;
     return launch_switch_tc2<KP>(prm, c->pair_clusters < cap ? c->pair_clusters : cap, s);
 }
@@ -791,25 +786,9 @@ int launch_switch(adafuse_ctx* ctx, int32_t layer_begin, int32_t n_layers,
         return e == cudaSuccess ? ADAFUSE_OK : cuda_fail(e, "switch launch");
     }
     if (kind == ADAFUSE_KERNEL_TCGEN05_FOLD) {
-        TcParams prm;
-        prm.pairs = ctx->d_pairs;
-        prm.tiles = ctx->d_tiles;
-        prm.maps = ctx->d_maps;
-        prm.blk = ctx->blk ? 1 : 0;
-        prm.t_begin = t0;
-        prm.t_end = t1;
-        prm.prev = prev;
-        prm.cur = cur;
-        prm.slots = slots;
-        prm.E = ctx->n_experts;
-        prm.s = ctx->scale;
-        prm.status = ctx->d_status;
-        prm.rebase = rebase ? 1 : 0;
-        prm.w0_maps = ctx->d_w0_maps;
-        prm.stall = ctx->stall_at;
-        ctx->stall_at = 0;
-        prm.dyn = 0;
-        prm.sched = nullptr;
+        // the folded kernel walks its tiles by a static stride
+        const TcParams prm =
+            tc_params(ctx, ctx->d_tiles, t0, t1, prev, cur, slots, rebase, false);
         const int64_t w0 = (int64_t)layer_begin * ctx->n_targets;
         const int64_t nw = (int64_t)n_layers * ctx->n_targets;
         const cudaError_t e =
