@@ -140,13 +140,19 @@ def test_pregate_empty_batch_is_a_noop():
     assert torch.all(routes == 7)
 
 
-@pytest.mark.parametrize("kernel,r", KERNEL_RANKS)
-def test_cuda_graph_capture_of_pregate_and_switch(kernel, r):
+@pytest.mark.parametrize("kernel,r,schedule",
+                         [(k, r, Bnd.ADAFUSE_SCHEDULE_AUTO) for (k, r) in KERNEL_RANKS] +
+                         [(TC2, 16, Bnd.ADAFUSE_SCHEDULE_DYNAMIC),
+                          (TC, 8, Bnd.ADAFUSE_SCHEDULE_STATIC)])
+def test_cuda_graph_capture_of_pregate_and_switch(kernel, r, schedule):
     """One decode step (pre-gate the token, switch prev -> cur, keep cur as the
     next prev) captured once and replayed gives the same W, bit for bit, as
-    the same calls made eagerly."""
+    the same calls made eagerly (both tile schedules: a dynamic launch leaves
+    its ticket counter at zero for the next replay)."""
     cfg, m1, s1 = _model(kernel, seed=9, r=r)
     _, m2, s2 = _model(kernel, seed=9, r=r)
+    s1.set_schedule(schedule)
+    s2.set_schedule(schedule)
     g = torch.Generator(device="cuda").manual_seed(5)
     T = 4
     hs = torch.randn((T, cfg.d), generator=g, device="cuda")
