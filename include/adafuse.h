@@ -188,7 +188,11 @@ ADAFUSE_API int adafuse_destroy(adafuse_ctx* ctx);
  * is a no-op.
  * Non-finite h gives an unspecified route (the switch rejects non-finite
  * gates).  One kernel launch on `stream` (a cudaStream_t, NULL = legacy
- * default stream). */
+ * default stream).  Batches of 64+ tokens with E == 8 and a 16-byte-aligned
+ * Wr bring Wr into each CTA by TMA tile loads behind a bounded wait: if
+ * those loads do not land within 1 s, the launch sets ADAFUSE_STATUS_TIMEOUT
+ * in the context's status word (adafuse_get_device_status) and writes no
+ * route. */
 ADAFUSE_API int adafuse_pregate(adafuse_ctx* ctx, const float* h, int64_t T, int64_t d,
                     const float* Wr, adafuse_route* route, void* stream);
 

@@ -620,17 +620,35 @@ int pregate_launch(adafuse_ctx* ctx, const float* h, int64_t T, int64_t d, const
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int E = ctx->n_experts;
     // Batches of 64+ tokens with up to 8 experts and d <= 4096: the
-    // token-group kernel (one warp per 4 tokens).  It computes the same bits
-    // as pregate_kernel, which takes every other case, so a token's route
-    // does not depend on which one ran.
+    // token-group kernel (a warp pair per 4 tokens).  It computes the same
+    // bits as pregate_kernel, which takes every other case, so a token's
+    // route does not depend on which one ran.
     const int64_t nch = ceil_div(d >> 2, 256);
     if (E <= 8 && nch <= kGroupMaxChunks && T >= kGroupMinTokens) {
         const size_t smem = group_smem_bytes(d);
         const int64_t ngroups = ceil_div(T, kGroupTokens);
         const unsigned grid = (unsigned)std::min<int64_t>(ngroups, (int64_t)ctx->sm_count);
+        // Wr staged by TMA tile loads when it is [d/4][32] floats (E == 8)
+        // at a 16-byte-aligned address; by the CTA's threads otherwise
+        CUtensorMap wr_map;
+        std::memset(&wr_map, 0, sizeof(wr_map));
+        int wr_tma = 0;
+        if (E == 8 && aligned16(Wr)) {
+            EncodeTiledFn enc = encode_tiled_fn();
+            const cuuint64_t dims[2] = {32, (cuuint64_t)(d >> 2)};
+            const cuuint64_t strides[1] = {128};
+            const cuuint32_t box[2] = {32, (cuuint32_t)kGroupWrBoxRows};
+            const cuuint32_t ones[2] = {1, 1};
+            wr_tma = enc != nullptr &&
+                     enc(&wr_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(Wr), dims,
+                         strides, box, ones, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+        }
         auto go = [&](auto kernel) {
             ensure_smem_attr(kernel, smem, ctx->device);
-            kernel<<<grid, kGroupThreads, smem, s>>>(h, T, d, Wr, E, k, slots, route, logits);
+            kernel<<<grid, kGroupThreads, smem, s>>>(h, T, d, Wr, E, k, slots, route, logits, wr_map,
+                                                     wr_tma, ctx->d_status);
         };
         switch (nch) {
             case 1: go(pregate_group_kernel<1>); break;

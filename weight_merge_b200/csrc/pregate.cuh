@@ -22,6 +22,8 @@
 // rule (lower index first) is exact.
 #pragma once
 
+#include <cuda.h>
+
 #include "common.cuh"
 #include "sm100_ptx.cuh"
 
@@ -204,8 +206,10 @@ pregate_kernel(const float* __restrict__ h, int64_t T, int64_t d, const float* _
 // kGroupTokens tokens: the even warp walks virtual warps 0..3, the odd warp
 // 4..7.  Per virtual warp and chunk index m a warp's lanes load the group's h
 // chunks (two such steps ahead of the arithmetic, in a ring of four register
-// slots), read Wr's rows from shared memory (staged once per CTA, shared by
-// the group's tokens) and accumulate; a reduce-scatter over the same lane
+// slots), read Wr's rows from shared memory (staged once per CTA, by TMA
+// tile loads with 128-byte swizzle when E == 8, else by the CTA's threads in
+// the same layout; shared by the group's tokens) and accumulate; a
+// reduce-scatter over the same lane
 // pairs as the xor tree (5 rounds, 31 shuffles for 32 (token, expert) sums)
 // then leaves lane L with token L / 8, expert L % 8 of that virtual warp.  The
 // even warp adds its four sums in order and hands the partial sum to the odd
@@ -213,6 +217,7 @@ pregate_kernel(const float* __restrict__ h, int64_t T, int64_t d, const float* _
 // alternating by group), which adds its own four in order: the same eight
 // additions as one warp walking all eight.  Four lanes of the odd warp then
 // run the four tokens' top-k tails side by side.
+
 // bar.sync on barrier `id` for `nthreads` threads (whole warps) of the CTA;
 // orders their shared-memory accesses like __syncthreads does for all.
 __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
@@ -225,24 +230,37 @@ constexpr int kGroupPairs = kGroupThreads / 64;
 constexpr int kGroupMaxChunks = 4;                 // d <= 256 * 4 * 4 = 4096
 constexpr int64_t kGroupMinTokens = 64;           // smaller batches: pregate_kernel
 
+constexpr int kGroupWrBoxRows = 256;                // chunks per Wr tile load (32 KB)
+
+// Wr in shared memory: chunk c (rows 4c..4c+3, experts 0..7) is 128 bytes,
+// its float4 f stored at slot c * 8 + (f ^ (c % 8)) -- the layout a TMA tile
+// load with 128-byte swizzle writes into a 1024-byte-aligned buffer -- so
+// lanes reading their own chunks 128 bytes apart hit distinct bank groups.
+// Whole 256-chunk boxes (zero past d).
 __host__ __device__ constexpr size_t group_wr_bytes(int64_t d) {
-    // Wr: one 4-row chunk (8 experts) per 9 float4 slots -- 8 of data, 1 of
-    // padding, so lanes reading their own chunks 144 bytes apart hit
-    // distinct bank groups
-    return (size_t)(d / 4) * 9 * 16;
+    return (size_t)((d / 4 + kGroupWrBoxRows - 1) / kGroupWrBoxRows) * kGroupWrBoxRows * 128;
 }
 __host__ __device__ constexpr size_t group_smem_bytes(int64_t d) {
-    // + the pairs' partial sums, two buffers of 32 lanes each
-    return group_wr_bytes(d) + (size_t)kGroupPairs * 2 * 32 * sizeof(float);
+    // 1024 bytes of alignment slack, Wr, the pairs' partial sums (two
+    // buffers of 32 lanes each) and the staging barrier
+    return 1024 + group_wr_bytes(d) + (size_t)kGroupPairs * 2 * 32 * sizeof(float) + 16;
 }
 
+// wr_map (used when wr_tma != 0): Wr viewed as [d / 4 chunks][32 floats],
+// box 32 x 256, 128-byte swizzle; E must be 8.  status receives
+// ADAFUSE_STATUS_TIMEOUT if those loads do not land within the wait limit.
 template <int NCH>
 __global__ void __launch_bounds__(kGroupThreads, 1)
 pregate_group_kernel(const float* __restrict__ h, int64_t T, int64_t d,
                      const float* __restrict__ Wr, int E, int k, int slots,
-                     int32_t* __restrict__ route, float* __restrict__ logits) {
-    extern __shared__ __align__(128) float4 wr_s[];
+                     int32_t* __restrict__ route, float* __restrict__ logits,
+                     const __grid_constant__ CUtensorMap wr_map, int wr_tma,
+                     int32_t* __restrict__ status) {
+    extern __shared__ __align__(1024) uint8_t group_smem_raw[];
+    float4* wr_s = reinterpret_cast<float4*>(
+        (reinterpret_cast<uintptr_t>(group_smem_raw) + 1023) & ~uintptr_t(1023));
     float* zpart_s = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(wr_s) + group_wr_bytes(d));
+    uint64_t* wr_bar = reinterpret_cast<uint64_t*>(zpart_s + kGroupPairs * 2 * 32);
     const int64_t nchunk = d >> 2;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int pair = warp >> 1, half = warp & 1;
@@ -282,10 +300,33 @@ pregate_group_kernel(const float* __restrict__ h, int64_t T, int64_t d,
     load_step(group_ptr(g_first), g_first, 0, ring[0]);
     load_step(group_ptr(g_first), g_first, 1, ring[1]);
 
-    // ---- Wr into shared memory: chunk c's rows 4c..4c+3 (experts 0..7, zero
-    // past E) as float4 slots c * 9 + 2 * q + (e / 4), kStageBatch loads in
-    // flight per thread before their stores
-    {
+    // ---- Wr into shared memory (the swizzled layout above): by TMA tile
+    // loads when the launch encoded a map (E == 8, Wr 16-byte aligned),
+    // otherwise by every thread, kStageBatch loads in flight before their
+    // stores (experts past E read as zero)
+    if (wr_tma) {
+        volatile int* no_abort = reinterpret_cast<volatile int*>(wr_bar + 1);   // stays 0
+        if (threadIdx.x == 0) {
+            *no_abort = 0;
+            sm100::mbar_init(wr_bar, 1);
+            sm100::fence_mbar_init();
+        }
+        __syncthreads();
+        const int nbox = (int)((nchunk + kGroupWrBoxRows - 1) / kGroupWrBoxRows);
+        if (threadIdx.x == 0) {
+            sm100::mbar_arrive_expect_tx(wr_bar, (uint32_t)nbox * kGroupWrBoxRows * 128u);
+            for (int b = 0; b < nbox; ++b)
+                sm100::tma_load_2d(reinterpret_cast<uint8_t*>(wr_s) + (size_t)b * kGroupWrBoxRows * 128,
+                                   &wr_map, 0, b * kGroupWrBoxRows, wr_bar);
+        }
+        const bool landed = sm100::mbar_wait_bounded(wr_bar, 0, no_abort, 1000000000ull);
+        // every thread of the CTA leaves together, or none does (the warp
+        // pairs meet at named barriers later)
+        if (__syncthreads_or(!landed)) {
+            if (threadIdx.x == 0) atomicOr(status, ADAFUSE_STATUS_TIMEOUT);
+            return;
+        }
+    } else {
         constexpr int kStageBatch = 8;
         const bool vec = E == 8 && (reinterpret_cast<uintptr_t>(Wr) & 15u) == 0;
         const int64_t total = nchunk * 8;
@@ -312,11 +353,11 @@ pregate_group_kernel(const float* __restrict__ h, int64_t T, int64_t d,
 #pragma unroll
             for (int u = 0; u < kStageBatch; ++u) {
                 const int64_t i = i0 + (int64_t)u * kGroupThreads;
-                if (i < total) wr_s[(i >> 3) * 9 + (i & 7)] = v[u];
+                if (i < total) wr_s[(i >> 3) * 8 + ((i & 7) ^ ((i >> 3) & 7))] = v[u];
             }
         }
+        __syncthreads();
     }
-    __syncthreads();
 
     const bool b16 = (lane & 16) != 0, b8 = (lane & 8) != 0, b4 = (lane & 4) != 0,
                b2 = (lane & 2) != 0, b1 = (lane & 1) != 0;
@@ -346,9 +387,10 @@ pregate_group_kernel(const float* __restrict__ h, int64_t T, int64_t d,
             }
             const int c = 32 * vw + lane + 256 * m;
             if (d_full || c < nch32) {
+                const int sw = c & 7;
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const float4 wa = wr_s[c * 9 + 2 * q], wb = wr_s[c * 9 + 2 * q + 1];
+                    const float4 wa = wr_s[c * 8 + ((2 * q) ^ sw)], wb = wr_s[c * 8 + ((2 * q + 1) ^ sw)];
                     const uint64_t w2[4] = {sm100::f32x2(wa.x, wa.y), sm100::f32x2(wa.z, wa.w),
                                             sm100::f32x2(wb.x, wb.y), sm100::f32x2(wb.z, wb.w)};
 #pragma unroll
