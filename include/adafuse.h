@@ -336,7 +336,9 @@ ADAFUSE_API int adafuse_pregate_topk(adafuse_ctx* ctx, const float* h, int64_t T
  * (INVALID_ARG above it; T == 0 is a no-op).  Two launches on `stream`: the
  * tokens' logits into a context-owned scratch of ADAFUSE_MAX_BATCH_TOKENS x E
  * fp32 (allocated at create), then the mean and the decision.  The scratch
- * is shared by the context's calls; calls on one stream are ordered. */
+ * is shared by the context's calls; calls on one stream are ordered.  If the
+ * first launch raises ADAFUSE_STATUS_TIMEOUT (see adafuse_pregate), the
+ * decision is taken from stale logits and must be discarded. */
 #define ADAFUSE_MAX_BATCH_TOKENS 4096
 ADAFUSE_API int adafuse_pregate_batch(adafuse_ctx* ctx, const float* h, int64_t T, int64_t d,
                                       const float* Wr, adafuse_route* route, void* stream);
