@@ -5,8 +5,9 @@
 // segment table and, per 128x128 W tile, applies
 //   W <- bf16_rne(W + sum_e c_e (B_e A_e)),  c_e = s (g_cur(e) - g_prev(e)).
 // The pages' ingredients map onto Blackwell like this:
-//   "segmented"       the tile table; each CTA takes a strided slice of it
-//                     (persistent grid, one CTA per SM);
+//   "segmented"       the tile table; each CTA takes its tiles by ticket in
+//                     table order or by a fixed stride (persistent grid, one
+//                     CTA per SM);
 //   "gather/concat"   per tile and selected expert, TMA fetches the expert's
 //                     B rows [row0, row0+128) x [0, r) and A columns
 //                     [col0, col0+128) x [0, r) straight from the stacked
@@ -15,9 +16,11 @@
 //                     TMA's out-of-bounds zero fill;
 //   "parallel GEMM"   one tcgen05.mma chain per expert into its own fp32 TMEM
 //                     accumulator (4 experts x 128 columns = all 512 columns);
-//   "in place"        W tiles go HBM -> smem (TMA, 128B swizzle) -> registers,
-//                     the epilogue adds sum_e c_e acc_e in fp32 and rounds once,
-//                     and TMA stores the tile back over itself;
+//   "in place"        W tiles go HBM -> smem (TMA, 128B swizzle; one operation
+//                     per tile where the weight's in is a multiple of 64) ->
+//                     registers, the epilogue adds sum_e c_e acc_e in fp32
+//                     (packed fp32 pairs) and rounds once, and TMA stores the
+//                     tile back over itself;
 //   "prefetch buffer" mbarrier-driven smem rings for W tiles and for operand
 //                     slices, filled ahead of use by a producer warp.
 // Warp roles: warp 0 W-tile producer (TMA), warp 1 TMEM owner
